@@ -1,0 +1,178 @@
+/*
+ * reatt.h -- C ABI of the B200 (sm_100a) ReAttention top-k span attention path.
+ *
+ * The operation (pages about "ReAttention: Training-Free Infinite Context with
+ * Finite Attention Scope", arXiv 2407.15176):
+ *   - arXiv abstract: position-agnostic top-k attention is taken before the
+ *     ordinary position-aware self-attention;
+ *   - research-map summary, "Approach": middle KV-cache segments are scored by
+ *     the dot product of the query with un-positioned keys, concatenated with
+ *     the global and local caches, and only then given positional embeddings;
+ *   - OpenReview discussion, "Decoding Phase" pseudocode: score = query .
+ *     key[global:-local]^T, top-k recall, concatenation global ++ recalled ++
+ *     local, then attention over that window;
+ *   - OpenReview discussion, NIAH settings: global 32, local 4096, segment 32.
+ * Fixed readings where the pages are silent: GQA scores sum q.k over the KV
+ * head's query heads (fp32 accumulation); a span's score is the max over its
+ * tokens (and over the C queries); ties prefer the lower span index; chosen
+ * spans keep ascending order; the window is global ++ chosen ++ local ++
+ * current; RoPE (rotate-half pairs (i, i+d/2), frequency base^(-2i/d)) at
+ * window positions 0..W-1, query c at W-C+c; causal softmax, scale 1/sqrt(d).
+ *
+ * Partition of the T cached tokens of one (batch, KV head):
+ *   global = [0, min(G,T)), local = [max(G, T-L), T), middle = [G, G+M),
+ *   M = max(0, T-G-L), NS = ceil(M/S) spans tiled from the left (the last one
+ *   may be short), k_eff = min(k, NS),
+ *   W = min(G,T) + (rows of the chosen spans) + (T - max(G, T-L) if T > G) + C,
+ *   Wmax = G + k*S + L + C  (an upper bound on W).
+ *
+ * Conventions for every entry point
+ *   - Layouts are contiguous row-major:
+ *       q            [B, Hq,  C,  d]     dtype
+ *       k/v cache    [B, Hkv, T,  d]     dtype, un-rotated (pre-RoPE)
+ *       k/v cur      [B, Hkv, C,  d]     dtype, un-rotated
+ *       span_scores  [B, Hkv, NS]        float32
+ *       sel          [B, Hkv, k]         int32, ascending span ids, -1 padded
+ *       k/v window   [B, Hkv, Wmax, d]   float32 (K rotated, V as is)
+ *       win_len      [B, Hkv]            int32
+ *       out          [B, Hq,  C,  d]     float32
+ *     Query head j reads KV head j / (Hq/Hkv).
+ *   - Every data pointer is a DEVICE pointer on the current device, 16-byte
+ *     aligned.  The caller owns all memory, including the workspace sized by
+ *     reatt_workspace_bytes(); the library allocates nothing and keeps no
+ *     state between calls (re-entrant on distinct workspaces).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous: results are valid once the stream has
+ *     reached that point.  Two calls that share a workspace must be ordered.
+ *   - Return value: REATT_OK, or an error code.  Arguments are checked on the
+ *     host before anything is enqueued; on an argument error nothing is
+ *     launched.  REATT_ECUDA reports a launch error (cudaGetLastError).
+ *     A kernel whose bounded wait gives up records REATT_ETIMEOUT in the
+ *     workspace status word, readable with reatt_workspace_status().
+ *     No C++ exception or abort crosses this interface.
+ */
+#ifndef REATT_H
+#define REATT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define REATT_API __attribute__((visibility("default")))
+#else
+#define REATT_API
+#endif
+
+/* Same type as cudaStream_t, declared here so this header needs no CUDA headers. */
+typedef struct CUstream_st *reatt_stream;
+
+typedef enum {
+    REATT_OK = 0,
+    REATT_EINVAL = 1,       /* null/misaligned pointer, bad or inconsistent size  */
+    REATT_EUNSUPPORTED = 2, /* valid request outside what the kernels implement    */
+    REATT_ECUDA = 3,        /* a CUDA call or kernel launch failed                  */
+    REATT_ETIMEOUT = 4      /* a kernel's bounded wait gave up (workspace status)   */
+} reatt_status;
+
+typedef enum { REATT_F32 = 0, REATT_BF16 = 1 } reatt_dtype;
+
+typedef struct {
+    int32_t B;          /* batch (independent sequences)                  >= 1 */
+    int32_t Hq;         /* query heads                                    >= 1 */
+    int32_t Hkv;        /* KV heads, Hq % Hkv == 0                        >= 1 */
+    int32_t d;          /* head width: 64 or 128                               */
+    int32_t C;          /* current (query) tokens: 1 = decode, >1 = prefill    */
+    int32_t G;          /* global tokens kept at the start                >= 0 */
+    int32_t L;          /* local tokens kept at the end                   >= 0 */
+    int32_t S;          /* span length                                    >= 1 */
+    int32_t k;          /* spans kept (top-k), 0 <= k <= 65536                 */
+    int32_t dtype;      /* reatt_dtype of q, caches and current tokens         */
+    int64_t T;          /* cached tokens, 0 <= T < 2^31                         */
+    double rope_base;   /* RoPE base (> 0, finite)                              */
+} reatt_dims;
+
+/* Text for a status code (static storage; never NULL). */
+REATT_API const char *reatt_status_string(int status);
+
+/* NS = ceil(max(0, T-G-L) / S).  EINVAL on bad dims or null output. */
+REATT_API int reatt_num_spans(const reatt_dims *dims, int64_t *num_spans);
+
+/* Wmax = G + k*S + L + C, the row capacity of the window buffers. */
+REATT_API int reatt_window_max(const reatt_dims *dims, int64_t *wmax);
+
+/* Bytes of device workspace any call with these dims may use (a multiple of
+ * 256).  The workspace holds a status word, split-K partials, top-k
+ * candidates, and, for reatt_step, the span scores and selection. */
+REATT_API int reatt_workspace_bytes(const reatt_dims *dims, size_t *bytes);
+
+/* Reads and clears the status word kept at the start of a workspace.  Waits
+ * for `stream`.  *status is REATT_OK or REATT_ETIMEOUT. */
+REATT_API int reatt_workspace_status(void *ws, int *status, reatt_stream stream);
+
+/*
+ * Span scoring (decoding pseudocode: score = query . key[global:-local]^T;
+ * research-map summary "Approach": un-positioned keys).
+ *   span_scores[b,h,s] = max over tokens t of span s and over queries c of
+ *                        sum_{j in group(h)} q[b,j,c,:] . k_cache[b,h,t,:]
+ * on un-rotated vectors, fp32 accumulation.  Writes B*Hkv*NS floats; no
+ * per-token score is ever stored.  ws: workspace of reatt_workspace_bytes().
+ */
+REATT_API int reatt_score_spans(const reatt_dims *dims, const void *q, const void *k_cache,
+                      float *span_scores, void *ws, reatt_stream stream);
+
+/*
+ * Top-k spans (decoding pseudocode: idx_recall = score.topk), per (b, h):
+ * the k_eff = min(k, NS) highest span_scores, ties to the lower span id,
+ * written in ascending span order (the cache order the window keeps);
+ * entries k_eff..k-1 are -1.  NaN scores are not supported.
+ */
+REATT_API int reatt_topk(const reatt_dims *dims, const float *span_scores, int32_t *sel, void *ws,
+               reatt_stream stream);
+
+/*
+ * Window construction (decoding pseudocode: concatenation global ++ recalled
+ * ++ local; "Approach": positional embedding applied after concatenation).
+ * For each (b, h): window rows = global ++ rows of the spans in sel (in the
+ * order given, which reatt_topk makes ascending) ++ local ++ the C current
+ * tokens.  K row p is rotated by RoPE at position p (fp32 arithmetic, angles
+ * reduced in fp64); V rows are copied.  Rows W..Wmax-1 are left untouched.
+ * win_len[b,h] = W.  sel must be laid out as reatt_topk writes it: the
+ * min(k, NS) chosen span ids in ascending order, then -1.  Other contents give
+ * unspecified rows, but every read stays inside the cache.
+ */
+REATT_API int reatt_gather_rope(const reatt_dims *dims, const void *k_cache, const void *v_cache,
+                      const void *k_cur, const void *v_cur, const int32_t *sel,
+                      float *k_win, float *v_win, int32_t *win_len, reatt_stream stream);
+
+/*
+ * Windowed attention (decoding pseudocode: flash_attention(query, key_recall,
+ * value_recall)).  Query c of head j is rotated at position W-C+c and attends
+ * window rows p <= W-C+c of KV head j/(Hq/Hkv) with softmax(q.k/sqrt(d)).
+ * k_win/v_win/win_len as written by reatt_gather_rope.  fp32 softmax and
+ * accumulation; split over the window with an in-kernel combine.
+ */
+REATT_API int reatt_attend(const reatt_dims *dims, const void *q, const float *k_win, const float *v_win,
+                 const int32_t *win_len, float *out, void *ws, reatt_stream stream);
+
+/*
+ * One whole step: score_spans -> topk -> attention over the virtual window.
+ * The window is never materialised: the attention reads global, chosen and
+ * local rows straight from the un-rotated cache (and the current tokens from
+ * k_cur/v_cur) and rotates them in registers.  Equal, up to fp32 rounding
+ * order, to reatt_score_spans + reatt_topk + reatt_gather_rope + reatt_attend.
+ * sel_out (nullable): receives the selection [B,Hkv,k].
+ * Appending the current tokens to the cache afterwards is the caller's job.
+ */
+REATT_API int reatt_step(const reatt_dims *dims, const void *q, const void *k_cache, const void *v_cache,
+               const void *k_cur, const void *v_cur, int32_t *sel_out, float *out, void *ws,
+               reatt_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* REATT_H */

@@ -1,0 +1,191 @@
+// Device helpers shared by the sm_100a kernels of the top-k span attention path.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "reatt.h"
+
+namespace reatt {
+
+// ----------------------------------------------------------------- geometry
+// Derived sizes of one call (host-computed, passed by value to kernels).
+struct Geom {
+    int B, Hq, Hkv, g, d, C, G, L, S, k;
+    int64_t T;
+    int64_t g_end;      // min(G, T)
+    int64_t loc_begin;  // max(G, T - L)
+    int64_t n_loc;      // T - loc_begin if T > loc_begin else 0
+    int64_t M;          // middle tokens
+    int64_t NS;         // spans
+    int64_t Wmax;       // G + k*S + L + C
+    double base;        // RoPE base
+    int dtype;          // reatt_dtype of q, caches, current tokens
+};
+
+// Workspace header: a status word kept at offset 0 of every workspace.
+constexpr size_t kWsHeader = 256;
+
+__device__ __forceinline__ void report_status(void *ws, uint32_t code)
+{
+    if (ws)
+        atomicMax(reinterpret_cast<unsigned int *>(ws), code);
+}
+
+// ----------------------------------------------------------------- numbers
+// bf16 pair (low half = lower address) -> two floats, exactly.
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// Order-preserving map float -> uint32 (larger float -> larger code; every
+// finite float and -inf maps above 0).
+__device__ __forceinline__ uint32_t order_code(float f)
+{
+    uint32_t u = __float_as_uint(f + 0.0f);   // -0 -> +0: equal floats, equal codes
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float order_decode(uint32_t c)
+{
+    return __uint_as_float((c & 0x80000000u) ? (c & 0x7fffffffu) : ~c);
+}
+
+// Element type tag: float (fp32) or bf16 stored as uint16_t.
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static constexpr int kBytes = 4;
+    static constexpr int kVec = 4;   // elements per 16-byte vector
+    __device__ __forceinline__ static void unpack(const uint4 &v, float (&o)[4])
+    {
+        o[0] = __uint_as_float(v.x);
+        o[1] = __uint_as_float(v.y);
+        o[2] = __uint_as_float(v.z);
+        o[3] = __uint_as_float(v.w);
+    }
+    __device__ __forceinline__ static float one(const float *p, int64_t i) { return p[i]; }
+};
+template <> struct Elem<uint16_t> {
+    static constexpr int kBytes = 2;
+    static constexpr int kVec = 8;
+    __device__ __forceinline__ static void unpack(const uint4 &v, float (&o)[8])
+    {
+        o[0] = bf16lo(v.x); o[1] = bf16hi(v.x);
+        o[2] = bf16lo(v.y); o[3] = bf16hi(v.y);
+        o[4] = bf16lo(v.z); o[5] = bf16hi(v.z);
+        o[6] = bf16lo(v.w); o[7] = bf16hi(v.w);
+    }
+    __device__ __forceinline__ static float one(const uint16_t *p, int64_t i)
+    {
+        return __uint_as_float(static_cast<uint32_t>(p[i]) << 16);
+    }
+};
+
+// 16-byte global load through the read-only path, not kept in L1.
+__device__ __forceinline__ uint4 ldg_stream(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// ----------------------------------------------------------------- RoPE
+// cos/sin of pos * base^(-2i/d).  The angle is formed and reduced modulo 2*pi
+// in fp64 (in units of pi), then evaluated in fp32 by sincospif on [-1, 1].
+__device__ __forceinline__ double rope_inv_freq_over_pi(int i, int d, double base)
+{
+    return pow(base, -2.0 * static_cast<double>(i) / static_cast<double>(d)) *
+           0.31830988618379067154;   // 1/pi
+}
+__device__ __forceinline__ void rope_cs(int64_t pos, double ifreq_over_pi, float &c, float &s)
+{
+    double x = static_cast<double>(pos) * ifreq_over_pi;   // angle / pi
+    x -= 2.0 * rint(0.5 * x);                                // now in [-1, 1]
+    sincospif(static_cast<float>(x), &s, &c);
+}
+
+// ----------------------------------------------------------------- mbarrier / bulk copy
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for the phase with the given parity to complete; gives up after
+// limit_ns of wall time and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > limit_ns)
+            return false;
+    }
+    return true;
+}
+// L2 policy: data read once (streamed K) is the first to be evicted.
+__device__ __forceinline__ uint64_t l2_evict_first_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+// Bulk (non-tensor) async copy global -> shared; completion is signalled on
+// the mbarrier as transaction bytes.  dst, src 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                          uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Bounded waits give up after this long (far above any legitimate wait).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+}  // namespace reatt

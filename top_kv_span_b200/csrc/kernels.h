@@ -1,0 +1,44 @@
+// Host-side launchers of the sm_100a kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace reatt {
+
+inline bool geo_is_bf16(const Geom &g) { return g.dtype == REATT_BF16; }
+
+int num_sms();
+
+// span scoring: scratch holds the fp32 summed queries when C > 1
+size_t score_spans_ws_bytes(const Geom &geo);
+cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, float *scores,
+                               void *ws, void *scratch, cudaStream_t st);
+
+// top-k: scratch holds per-slice candidates when NS is large; zero_words
+// (nullable) are cleared by the first CTA (used to reset attention tickets)
+size_t topk_ws_bytes(const Geom &geo);
+cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void *scratch,
+                        uint32_t *zero_words, int nzero, cudaStream_t st);
+
+cudaError_t launch_gather_rope(const Geom &geo, const void *kc, const void *vc, const void *kcur,
+                               const void *vcur, const int32_t *sel, float *kw, float *vw,
+                               int32_t *win_len, cudaStream_t st);
+
+struct AttnPlan {
+    int QB, nqb, nsplit;
+};
+AttnPlan attn_plan(const Geom &geo);
+// bytes of tickets (256-aligned, reported separately) + split-K partials
+size_t attend_ws_bytes(const Geom &geo, size_t *ticket_bytes);
+// virt = true: keys/values read from the un-rotated cache through sel;
+// virt = false: from the materialised fp32 window (kw, vw, win_len).
+cudaError_t launch_attend(const Geom &geo, const void *q, const float *kw, const float *vw,
+                          const int32_t *win_len, const void *kc, const void *vc,
+                          const void *kcur, const void *vcur, const int32_t *sel, float *out,
+                          void *scratch, bool virt, cudaStream_t st);
+
+}  // namespace reatt

@@ -1,0 +1,186 @@
+"""Thin ctypes binding of ``libreatt.so`` (the C ABI in ``include/reatt.h``).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Functions keep the C names; tensors are passed as device pointers,
+the stream defaults to torch's current stream.  Missing library -> ImportError
+(there is no fallback of any kind).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libreatt.so")
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT = 0, 1, 2, 3, 4
+F32, BF16 = 0, 1
+
+EXPORTS = ["reatt_status_string", "reatt_num_spans", "reatt_window_max", "reatt_workspace_bytes",
+           "reatt_workspace_status", "reatt_score_spans", "reatt_topk", "reatt_gather_rope",
+           "reatt_attend", "reatt_step"]
+
+
+class reatt_dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("C", ctypes.c_int32), ("G", ctypes.c_int32),
+                ("L", ctypes.c_int32), ("S", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("T", ctypes.c_int64), ("rope_base", ctypes.c_double)]
+
+
+class ReattError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m top_kv_span_b200.build` "
+                      "(nvcc, sm_100a); there is no fallback path")
+
+lib = ctypes.CDLL(LIB_PATH)
+_vp, _dp = ctypes.c_void_p, ctypes.POINTER(reatt_dims)
+lib.reatt_status_string.restype = ctypes.c_char_p
+lib.reatt_status_string.argtypes = [ctypes.c_int]
+lib.reatt_num_spans.argtypes = [_dp, ctypes.POINTER(ctypes.c_int64)]
+lib.reatt_window_max.argtypes = [_dp, ctypes.POINTER(ctypes.c_int64)]
+lib.reatt_workspace_bytes.argtypes = [_dp, ctypes.POINTER(ctypes.c_size_t)]
+lib.reatt_workspace_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int), _vp]
+lib.reatt_score_spans.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp]
+lib.reatt_topk.argtypes = [_dp, _vp, _vp, _vp, _vp]
+lib.reatt_gather_rope.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.reatt_attend.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.reatt_step.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+for _name in EXPORTS[1:]:
+    getattr(lib, _name).restype = ctypes.c_int
+
+
+def status_string(code: int) -> str:
+    return lib.reatt_status_string(int(code)).decode()
+
+
+def make_dims(B, Hq, Hkv, d, C, T, G, L, S, k, dtype, rope_base) -> reatt_dims:
+    if isinstance(dtype, str):
+        dtype = F32 if dtype == "f32" else BF16
+    elif isinstance(dtype, torch.dtype):
+        dtype = F32 if dtype == torch.float32 else BF16
+    return reatt_dims(int(B), int(Hq), int(Hkv), int(d), int(C), int(G), int(L), int(S), int(k),
+                      int(dtype), int(T), float(rope_base))
+
+
+def dims_of(w, **override) -> reatt_dims:
+    """Dims of a ``workloads.Workload`` (fields may be overridden)."""
+    f = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, C=w.C, T=w.T, G=w.G, L=w.L, S=w.S, k=w.k,
+             dtype=w.dtype, rope_base=w.rope_base)
+    f.update(override)
+    return make_dims(**f)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc, where):
+    if rc != OK:
+        raise ReattError(rc, where)
+
+
+def reatt_num_spans(dims) -> int:
+    v = ctypes.c_int64()
+    _check(lib.reatt_num_spans(ctypes.byref(dims), ctypes.byref(v)), "reatt_num_spans")
+    return v.value
+
+
+def reatt_window_max(dims) -> int:
+    v = ctypes.c_int64()
+    _check(lib.reatt_window_max(ctypes.byref(dims), ctypes.byref(v)), "reatt_window_max")
+    return v.value
+
+
+def reatt_workspace_bytes(dims) -> int:
+    v = ctypes.c_size_t()
+    _check(lib.reatt_workspace_bytes(ctypes.byref(dims), ctypes.byref(v)),
+           "reatt_workspace_bytes")
+    return v.value
+
+
+def reatt_workspace_status(ws, stream=None) -> int:
+    v = ctypes.c_int()
+    _check(lib.reatt_workspace_status(_ptr(ws), ctypes.byref(v), _stream(stream)),
+           "reatt_workspace_status")
+    return v.value
+
+
+def reatt_score_spans(dims, q, k_cache, span_scores, ws, stream=None, check=True):
+    rc = lib.reatt_score_spans(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(span_scores),
+                               _ptr(ws), _stream(stream))
+    if check:
+        _check(rc, "reatt_score_spans")
+    return rc
+
+
+def reatt_topk(dims, span_scores, sel, ws, stream=None, check=True):
+    rc = lib.reatt_topk(ctypes.byref(dims), _ptr(span_scores), _ptr(sel), _ptr(ws),
+                        _stream(stream))
+    if check:
+        _check(rc, "reatt_topk")
+    return rc
+
+
+def reatt_gather_rope(dims, k_cache, v_cache, k_cur, v_cur, sel, k_win, v_win, win_len,
+                      stream=None, check=True):
+    rc = lib.reatt_gather_rope(ctypes.byref(dims), _ptr(k_cache), _ptr(v_cache), _ptr(k_cur),
+                               _ptr(v_cur), _ptr(sel), _ptr(k_win), _ptr(v_win), _ptr(win_len),
+                               _stream(stream))
+    if check:
+        _check(rc, "reatt_gather_rope")
+    return rc
+
+
+def reatt_attend(dims, q, k_win, v_win, win_len, out, ws, stream=None, check=True):
+    rc = lib.reatt_attend(ctypes.byref(dims), _ptr(q), _ptr(k_win), _ptr(v_win), _ptr(win_len),
+                          _ptr(out), _ptr(ws), _stream(stream))
+    if check:
+        _check(rc, "reatt_attend")
+    return rc
+
+
+def reatt_step(dims, q, k_cache, v_cache, k_cur, v_cur, sel_out, out, ws, stream=None,
+               check=True):
+    rc = lib.reatt_step(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_cur),
+                        _ptr(v_cur), _ptr(sel_out), _ptr(out), _ptr(ws), _stream(stream))
+    if check:
+        _check(rc, "reatt_step")
+    return rc
+
+
+# ----------------------------------------------------------------- convenience
+def alloc_outputs(dims, device="cuda"):
+    """Caller-side buffers for one call of every entry point (torch allocates)."""
+    NS = reatt_num_spans(dims)
+    Wmax = reatt_window_max(dims)
+    BH = dims.B * dims.Hkv
+    ws_bytes = reatt_workspace_bytes(dims)
+    return dict(
+        span_scores=torch.empty((dims.B, dims.Hkv, NS), dtype=torch.float32, device=device),
+        sel=torch.empty((dims.B, dims.Hkv, dims.k), dtype=torch.int32, device=device),
+        k_win=torch.zeros((dims.B, dims.Hkv, Wmax, dims.d), dtype=torch.float32, device=device),
+        v_win=torch.zeros((dims.B, dims.Hkv, Wmax, dims.d), dtype=torch.float32, device=device),
+        win_len=torch.empty((dims.B, dims.Hkv), dtype=torch.int32, device=device),
+        out=torch.empty((dims.B, dims.Hq, dims.C, dims.d), dtype=torch.float32, device=device),
+        ws=torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=device),
+    )
