@@ -52,23 +52,30 @@ int make_geom(const reatt_dims *d, Geom *g)
     g->Wmax = int64_t(d->G) + int64_t(d->k) * d->S + d->L + d->C;
     g->base = d->rope_base;
     g->dtype = d->dtype;
+    for (int i = 0; i < 64; ++i) {
+        g->rope_hi[i] = g->rope_lo[i] = 0.f;
+        if (i < d->d / 2) {
+            const double f = pow(d->rope_base, -2.0 * i / double(d->d)) / M_PI;
+            g->rope_hi[i] = float(f);
+            g->rope_lo[i] = float(f - double(g->rope_hi[i]));
+        }
+    }
     return REATT_OK;
 }
 
 // Workspace layout: [status header][attention tickets][attention partials]
-// [top-k candidates][summed queries (C > 1)][span scores][selection].
+// [top-k candidates][summed queries (C > 1)][span scores][selection][RoPE table].
 struct WsPlan {
-    size_t ticket, ticket_bytes, part, topk, qsum, scores, sel, total;
+    size_t ticket, ticket_bytes, topk, qsum, scores, sel, tab, total;
 };
 WsPlan ws_plan(const Geom &g)
 {
     WsPlan p;
     size_t off = kWsHeader;
-    size_t tb = 0;
-    const size_t attn = attend_ws_bytes(g, &tb);
+    size_t tb = 0, mo = 0;
+    const size_t attn = attend_ws_bytes(g, &tb, &mo);
     p.ticket = off;
     p.ticket_bytes = tb;
-    p.part = off + tb;
     off = up256(off + attn);
     p.topk = off;
     off = up256(off + topk_ws_bytes(g));
@@ -78,6 +85,8 @@ WsPlan ws_plan(const Geom &g)
     off = up256(off + size_t(g.B) * g.Hkv * g.NS * sizeof(float));
     p.sel = off;
     off = up256(off + size_t(g.B) * g.Hkv * g.k * sizeof(int32_t));
+    p.tab = off;
+    off = up256(off + rope_table_bytes(g));
     p.total = off;
     return p;
 }
@@ -175,7 +184,8 @@ int reatt_topk(const reatt_dims *dims, const float *span_scores, int32_t *sel, v
     if (!aligned16(sel) || !aligned16(ws) || !aligned16(span_scores)) return REATT_EINVAL;
     const WsPlan p = ws_plan(g);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return cuda_status(launch_topk(g, span_scores, sel, at(ws, p.topk), nullptr, 0, st));
+    return cuda_status(
+        launch_topk(g, span_scores, sel, at(ws, p.topk), nullptr, 0, nullptr, st));
 }
 
 int reatt_gather_rope(const reatt_dims *dims, const void *k_cache, const void *v_cache,
@@ -212,7 +222,8 @@ int reatt_attend(const reatt_dims *dims, const void *q, const float *k_win, cons
     cudaError_t e = cudaMemsetAsync(at(ws, p.ticket), 0, p.ticket_bytes, st);
     if (e != cudaSuccess) return REATT_ECUDA;
     return cuda_status(launch_attend(g, q, k_win, v_win, win_len, nullptr, nullptr, nullptr,
-                                     nullptr, nullptr, out, at(ws, p.ticket), false, st));
+                                     nullptr, nullptr, nullptr, out, at(ws, p.ticket), ws, false,
+                                     st));
 }
 
 int reatt_step(const reatt_dims *dims, const void *q, const void *k_cache, const void *v_cache,
@@ -233,12 +244,13 @@ int reatt_step(const reatt_dims *dims, const void *q, const void *k_cache, const
     int32_t *sel = sel_out ? sel_out : reinterpret_cast<int32_t *>(at(ws, p.sel));
     cudaError_t e = launch_score_spans(g, q, k_cache, scores, ws, at(ws, p.qsum), st);
     if (e != cudaSuccess) return REATT_ECUDA;
-    // the top-k launch also clears the attention tickets
+    // the top-k launch also clears the attention tickets and fills the RoPE table
+    float2 *tab = reinterpret_cast<float2 *>(at(ws, p.tab));
     e = launch_topk(g, scores, sel, at(ws, p.topk), reinterpret_cast<uint32_t *>(at(ws, p.ticket)),
-                    int(p.ticket_bytes / sizeof(uint32_t)), st);
+                    int(p.ticket_bytes / sizeof(uint32_t)), tab, st);
     if (e != cudaSuccess) return REATT_ECUDA;
     return cuda_status(launch_attend(g, q, nullptr, nullptr, nullptr, k_cache, v_cache, k_cur,
-                                     v_cur, sel, out, at(ws, p.ticket), true, st));
+                                     v_cur, sel, tab, out, at(ws, p.ticket), ws, true, st));
 }
 
 }  // extern "C"

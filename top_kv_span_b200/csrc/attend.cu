@@ -21,6 +21,8 @@
 // ticket, no waiting) merges them and writes the output.
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -30,7 +32,9 @@ namespace {
 
 constexpr int kAttnThreads = 256;
 constexpr int kKT = 64;                 // keys per tile
-constexpr int kTargetCtas = 296;        // 2 x 148 SMs: split-K target
+constexpr int kTargetCtas = 296;        // tile kernel: ~2 CTAs per SM (148 SMs)
+constexpr int kDecodeCtas = 148;        // decode kernels: ~1 CTA per SM
+constexpr int kMinSplitKeys = 128;      // keys per split at least
 
 struct WinMap {
     int64_t g_end, loc_begin, n_loc, nsel_rows, W;
@@ -83,13 +87,12 @@ gather_rope_kernel(Geom geo, const T *__restrict__ kc, const T *__restrict__ vc,
                    int32_t *__restrict__ win_len)
 {
     constexpr int V = Elem<T>::kVec, HV = D / 2 / V;   // vectors per half row
-    __shared__ double ifreq[D / 2];
+    __shared__ float2 freq[D / 2];
     const int64_t bh = blockIdx.y;
     const int32_t *sel_bh = sel + bh * geo.k;
     const WinMap m = make_winmap(geo, sel_bh);
-    for (int i = threadIdx.x; i < D / 2; i += blockDim.x)
-        ifreq[i] = rope_inv_freq_over_pi(i, D, geo.base);
     if (blockIdx.x == 0 && threadIdx.x == 0) win_len[bh] = int32_t(m.W);
+    if (threadIdx.x < D / 2) freq[threadIdx.x] = make_float2(geo.rope_hi[threadIdx.x], geo.rope_lo[threadIdx.x]);
     __syncthreads();
 
     const int64_t row0 = int64_t(blockIdx.x) * kGatherRows;
@@ -113,45 +116,835 @@ gather_rope_kernel(Geom geo, const T *__restrict__ kc, const T *__restrict__ vc,
         Elem<T>::unpack(*reinterpret_cast<const uint4 *>(vr + D / 2 + v * V), vhi);
         float *ko = kw + (bh * geo.Wmax + p) * D;
         float *vo = vw + (bh * geo.Wmax + p) * D;
+        float rl[V], rh[V];
 #pragma unroll
         for (int e = 0; e < V; ++e) {
             const int i = v * V + e;
             float c, sn;
-            rope_cs(p, ifreq[i], c, sn);
-            ko[i] = klo[e] * c - khi[e] * sn;
-            ko[i + D / 2] = khi[e] * c + klo[e] * sn;
-            vo[i] = vlo[e];
-            vo[i + D / 2] = vhi[e];
+            rope_cs(p, freq[i].x, freq[i].y, c, sn);
+            rl[e] = klo[e] * c - khi[e] * sn;
+            rh[e] = khi[e] * c + klo[e] * sn;
+        }
+#pragma unroll
+        for (int e = 0; e < V; e += 4) {
+            const int i = v * V + e;
+            *reinterpret_cast<float4 *>(ko + i) = make_float4(rl[e], rl[e + 1], rl[e + 2], rl[e + 3]);
+            *reinterpret_cast<float4 *>(ko + i + D / 2) = make_float4(rh[e], rh[e + 1], rh[e + 2], rh[e + 3]);
+            *reinterpret_cast<float4 *>(vo + i) = make_float4(vlo[e], vlo[e + 1], vlo[e + 2], vlo[e + 3]);
+            *reinterpret_cast<float4 *>(vo + i + D / 2) = make_float4(vhi[e], vhi[e + 1], vhi[e + 2], vhi[e + 3]);
         }
     }
 }
 
 // ---------------------------------------------------------------- attention
-template <int D, int QB>
-struct AttnSmem {
-    static constexpr size_t kQ = size_t(QB) * D * 4;
-    static constexpr size_t kK = size_t(kKT) * (D + 1) * 4;
-    static constexpr size_t kV = size_t(kKT) * D * 4;
-    static constexpr size_t kP = size_t(QB) * kKT * 4;
-    static constexpr size_t kRow = size_t(QB) * 4 * 3;   // m, l, corr
-    static constexpr size_t kF = size_t(D / 2) * 8;
-    static constexpr size_t kTotal = kQ + kK + kV + kP + kRow + kF + 64;
+struct AttnArgs {
+    const void *q;
+    const int32_t *sel;       // virtual window
+    const int32_t *win_len;   // materialised window
+    const float2 *tab;        // virtual window: RoPE cos/sin [Wmax][D/2]
+    float *out;
+    float *part_acc;          // [BH][nqb][nsplit][QB][D]
+    float2 *part_ml;          // [BH][nqb][nsplit][QB] (max, sum)
+    uint32_t *ticket;         // [BH][nqb]
+    int nqb, nsplit;
 };
 
-// Key/value row source for the two attention variants.
+__device__ __forceinline__ WinMap attn_winmap(const Geom &geo, const AttnArgs &a, bool virt,
+                                              int64_t bh, const int32_t *sel_bh)
+{
+    if (virt) return make_winmap(geo, sel_bh);
+    WinMap m;
+    m.g_end = m.loc_begin = m.n_loc = m.nsel_rows = 0;
+    const int64_t wl = a.win_len[bh];   // caller data: keep every read inside the window
+    m.W = wl < geo.C ? geo.C : (wl > geo.Wmax ? geo.Wmax : wl);
+    return m;
+}
+
+// Key range of one split (whole multiples of `gran` keys), clipped by the
+// causal limit of the block's last query row.
+__device__ __forceinline__ void split_range(const Geom &geo, int64_t W, int nsplit, int split,
+                                            int r0, int nrows, int gran, int64_t &kbeg,
+                                            int64_t &kend)
+{
+    int64_t chunk = (W + nsplit - 1) / nsplit;
+    chunk = (chunk + gran - 1) / gran * gran;
+    kbeg = int64_t(split) * chunk;
+    kend = kbeg + chunk;
+    if (kend > W) kend = W;
+    const int last_row = r0 + nrows - 1;
+    const int c_max = (last_row / geo.C == r0 / geo.C) ? last_row % geo.C : geo.C - 1;
+    const int64_t lim = W - geo.C + c_max + 1;
+    if (kend > lim) kend = lim;
+}
+
+// End of a CTA's work: its (max, sum, acc) per row sit in shared memory.  With
+// one split the output is written directly; otherwise the split's partial
+// goes to the workspace and the last CTA of (bh, qb) to finish (atomic ticket,
+// no waiting) merges all splits.  `scratch` holds >= nsplit*QB floats.
+template <int D, int QB>
+__device__ void split_finish(const Geom &geo, const AttnArgs &a, int64_t bh, int qb, int split,
+                             int nrows, const float *s_m, const float *s_l, const float *s_acc,
+                             float *scratch, int *is_last)
+{
+    constexpr int D4 = D / 4;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthr = blockDim.x;
+    const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv), r0 = qb * QB;
+    auto out4 = [&](int rr) {
+        const int r = r0 + rr, j = h * geo.g + r / geo.C, c = r % geo.C;
+        return reinterpret_cast<float4 *>(a.out + ((int64_t(b) * geo.Hq + j) * geo.C + c) * D);
+    };
+    if (a.nsplit == 1) {
+        for (int x = tid; x < nrows * D4; x += nthr) {
+            const int rr = x / D4, d4 = x % D4;
+            const float il = 1.f / s_l[rr];
+            const float4 v = reinterpret_cast<const float4 *>(s_acc)[rr * D4 + d4];
+            out4(rr)[d4] = make_float4(v.x * il, v.y * il, v.z * il, v.w * il);
+        }
+        return;
+    }
+    const int64_t pbase = (bh * a.nqb + qb) * a.nsplit;
+    float4 *pacc = reinterpret_cast<float4 *>(a.part_acc + (pbase + split) * int64_t(QB) * D);
+    for (int x = tid; x < nrows * D4; x += nthr)
+        pacc[x] = reinterpret_cast<const float4 *>(s_acc)[x];
+    for (int rr = tid; rr < nrows; rr += nthr)
+        a.part_ml[(pbase + split) * QB + rr] = make_float2(s_m[rr], s_l[rr]);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const uint32_t prev = atomicAdd(&a.ticket[bh * a.nqb + qb], 1u);
+        *is_last = prev == uint32_t(a.nsplit - 1);
+    }
+    __syncthreads();
+    if (!*is_last) return;
+    __threadfence();
+    // w[s][r] = exp2(m_s - M_r) / sum_s' l_s' exp2(m_s' - M_r)
+    float *wgt = scratch;
+    const float2 *ml = a.part_ml + pbase * QB;
+    for (int x = tid; x < a.nsplit * QB; x += nthr) {
+        const int rr = x % QB;
+        wgt[x] = rr < nrows ? __ldcg(&ml[x].x) : -INFINITY;
+    }
+    __syncthreads();
+    for (int rr = warp; rr < nrows; rr += nthr / 32) {
+        float mx = -INFINITY;
+        for (int s = lane; s < a.nsplit; s += 32) mx = fmaxf(mx, wgt[s * QB + rr]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float den = 0.f;
+        for (int s = lane; s < a.nsplit; s += 32) {
+            const float ms = wgt[s * QB + rr];
+            const float w = ms == -INFINITY ? 0.f : exp2f(ms - mx);
+            den += w * __ldcg(&ml[s * QB + rr].y);
+            wgt[s * QB + rr] = w;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        const float iden = 1.f / den;
+        __syncwarp();
+        for (int s = lane; s < a.nsplit; s += 32) wgt[s * QB + rr] *= iden;
+    }
+    __syncthreads();
+    const float4 *all = reinterpret_cast<const float4 *>(a.part_acc + pbase * int64_t(QB) * D);
+    for (int x = tid; x < nrows * D4; x += nthr) {
+        const int rr = x / D4;
+        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int s = 0; s < a.nsplit; ++s) {
+            const float w = wgt[s * QB + rr];
+            const float4 v = __ldcg(all + int64_t(s) * QB * D4 + x);
+            z.x = fmaf(w, v.x, z.x);
+            z.y = fmaf(w, v.y, z.y);
+            z.z = fmaf(w, v.z, z.z);
+            z.w = fmaf(w, v.w, z.w);
+        }
+        out4(rr)[x % D4] = z;
+    }
+    if (tid == 0) a.ticket[bh * a.nqb + qb] = 0u;   // ready for the next call
+}
+
+// Rotated, pre-scaled query element pair (i, i + D/2) of block row rr:
+// log2(e)/sqrt(d) folds the softmax scale so logits live in the log2 domain.
+template <typename T, int D>
+__device__ __forceinline__ void query_pair(const Geom &geo, const float2 *freq, const void *q,
+                                           int b, int h, int r, int64_t qpos0, int i, float &lo,
+                                           float &hi)
+{
+    const float qscale = 1.4426950408889634f * rsqrtf(float(D));
+    const int j = h * geo.g + r / geo.C, c = r % geo.C;
+    const T *qr = static_cast<const T *>(q) + ((int64_t(b) * geo.Hq + j) * geo.C + c) * D;
+    const float x0 = Elem<T>::one(qr, i), x1 = Elem<T>::one(qr, i + D / 2);
+    float cs, sn;
+    rope_cs(qpos0 + c, freq[i].x, freq[i].y, cs, sn);
+    lo = (x0 * cs - x1 * sn) * qscale;
+    hi = (x1 * cs + x0 * sn) * qscale;
+}
+
+// ---------------------------------------------------------------- decode attention
+// For few query rows per KV head (R = g*C <= 8, padded to RP): one warp walks
+// keys in batches of KB = 32/RP.  Lane l owns the RoPE pairs PD*l .. PD*l+PD-1
+// (PD = D/64) and their partners at +D/2, so a key row is rotated in
+// registers.  Per batch the KB x RP partial dot products are folded by one
+// transposed shuffle reduction (lane i ends with pair (key i/RP, row i%RP)),
+// softmax is online per row, and P.V accumulates in registers.  No shared
+// memory is touched until the warps of the CTA merge their states.
+// Raw (unconverted) words of one lane's PD elements of a row: loaded early,
+// converted only when the batch is computed, so loads of the next keys are in
+// flight meanwhile.
+template <typename T, int PD> struct PairRaw;
+template <> struct PairRaw<uint16_t, 2> {
+    uint32_t w;
+    __device__ __forceinline__ void ld(const uint16_t *p)
+    {
+        w = __ldg(reinterpret_cast<const unsigned int *>(p));
+    }
+    __device__ __forceinline__ void lds(const uint8_t *p) { w = *reinterpret_cast<const uint32_t *>(p); }
+    __device__ __forceinline__ void get(float (&o)[2]) const
+    {
+        o[0] = bf16lo(w);
+        o[1] = bf16hi(w);
+    }
+};
+template <> struct PairRaw<uint16_t, 1> {
+    uint32_t w;
+    __device__ __forceinline__ void ld(const uint16_t *p)
+    {
+        w = __ldg(reinterpret_cast<const unsigned short *>(p));
+    }
+    __device__ __forceinline__ void lds(const uint8_t *p) { w = *reinterpret_cast<const uint16_t *>(p); }
+    __device__ __forceinline__ void get(float (&o)[1]) const { o[0] = __uint_as_float(w << 16); }
+};
+template <> struct PairRaw<float, 2> {
+    float2 w;
+    __device__ __forceinline__ void ld(const float *p) { w = __ldg(reinterpret_cast<const float2 *>(p)); }
+    __device__ __forceinline__ void lds(const uint8_t *p) { w = *reinterpret_cast<const float2 *>(p); }
+    __device__ __forceinline__ void get(float (&o)[2]) const
+    {
+        o[0] = w.x;
+        o[1] = w.y;
+    }
+};
+template <> struct PairRaw<float, 1> {
+    float w;
+    __device__ __forceinline__ void ld(const float *p) { w = __ldg(p); }
+    __device__ __forceinline__ void lds(const uint8_t *p) { w = *reinterpret_cast<const float *>(p); }
+    __device__ __forceinline__ void get(float (&o)[1]) const { o[0] = w; }
+};
+
+// Window row p -> element offset of its K/V row: cache rows at (bh*T + s)*D,
+// current token c at a separate base (flag bit 62 set), in 32-bit index math.
+__device__ __forceinline__ int64_t win_row_offset(const Geom &geo, const WinMap &m,
+                                                  const int32_t *sel_bh, int64_t bh, int p, int D)
+{
+    const int g_end = int(m.g_end), nsel = int(m.nsel_rows), nloc = int(m.n_loc);
+    int s;
+    if (p < g_end) {
+        s = p;
+    } else if (p - g_end < nsel) {
+        const int q = p - g_end, j = q / geo.S, off = q - j * geo.S;
+        int sp = sel_bh[j];
+        sp = sp < 0 ? 0 : (sp >= int(geo.NS) ? int(geo.NS) - 1 : sp);
+        s = geo.G + sp * geo.S + off;
+        if (s >= int(geo.T)) s = int(geo.T) - 1;
+    } else if (p - g_end - nsel < nloc) {
+        s = int(m.loc_begin) + (p - g_end - nsel);
+    } else {
+        const int c = p - g_end - nsel - nloc;
+        return (int64_t(1) << 62) | ((bh * geo.C + c) * D);
+    }
+    return (bh * geo.T + s) * D;
+}
+
+constexpr int kDecWarps = 8;
+
+template <typename T, int D, int RP, bool VIRT>
+__global__ void __launch_bounds__(kDecWarps * 32, 2)
+attend_decode_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__restrict__ vc,
+                     const T *__restrict__ kcur, const T *__restrict__ vcur,
+                     const float *__restrict__ kw, const float *__restrict__ vw)
+{
+    constexpr int PD = D / 64;            // RoPE pairs per lane
+    constexpr int KB = 32 / RP;           // keys per batch
+    using RowT = typename std::conditional<VIRT, T, float>::type;
+    __shared__ float s_m[kDecWarps][RP], s_l[kDecWarps][RP];
+    __shared__ __align__(16) float s_acc[kDecWarps][RP][D];
+    __shared__ float f_m[RP], f_l[RP];
+    __shared__ float2 freq[D / 2];
+    __shared__ int is_last;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid < D / 2) freq[tid] = make_float2(geo.rope_hi[tid], geo.rope_lo[tid]);
+    __syncthreads();
+    const int split = blockIdx.x;
+    const int64_t bh = blockIdx.z;
+    const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv);
+    const int nrows = geo.g * geo.C;     // <= RP (one query block)
+    const int32_t *sel_bh = VIRT ? a.sel + bh * geo.k : nullptr;
+    const WinMap m = attn_winmap(geo, a, VIRT, bh, sel_bh);
+    const int64_t W = m.W, qpos0 = W - geo.C;
+    int64_t kbeg, kend;
+    split_range(geo, W, a.nsplit, split, 0, nrows, 32, kbeg, kend);
+
+    // this lane's query pairs for every row (zero for padded rows)
+    float qlo[RP][PD], qhi[RP][PD];
+#pragma unroll
+    for (int r = 0; r < RP; ++r)
+#pragma unroll
+        for (int e = 0; e < PD; ++e) {
+            qlo[r][e] = qhi[r][e] = 0.f;
+            if (r < nrows)
+                query_pair<T, D>(geo, freq, a.q, b, h, r, qpos0, PD * lane + e, qlo[r][e], qhi[r][e]);
+        }
+    // causal limit of this lane's logit row (lane % RP) and of every row
+    const int my_r = lane % RP;
+    const int64_t my_lim = my_r < nrows ? qpos0 + my_r % geo.C : -1;
+
+    float mrow[RP], lrow[RP], alo[RP][PD], ahi[RP][PD];
+#pragma unroll
+    for (int r = 0; r < RP; ++r) {
+        mrow[r] = -INFINITY;
+        lrow[r] = 0.f;
+#pragma unroll
+        for (int e = 0; e < PD; ++e) alo[r][e] = ahi[r][e] = 0.f;
+    }
+    float m_own = -INFINITY;
+
+    constexpr int NB = KB <= 8 ? 2 : 1;   // batches whose loads go out together
+    constexpr int KI = NB * KB;             // keys per warp iteration (<= 32)
+    for (int64_t pi = kbeg + int64_t(warp) * KI; pi < kend; pi += int64_t(kDecWarps) * KI) {
+        // lane kk < KI resolves the row of key pi + kk once; the others take
+        // it by shuffle
+        int64_t my_off = -1;
+        if (lane < KI && pi + lane < kend) {
+            if (VIRT) my_off = win_row_offset(geo, m, sel_bh, bh, int(pi + lane), D);
+            else my_off = (bh * geo.Wmax + pi + lane) * D;
+        }
+        PairRaw<RowT, PD> rkl[KI], rkh[KI], rvl[KI], rvh[KI];
+#pragma unroll
+        for (int kk = 0; kk < KI; ++kk) {
+            const int64_t off = __shfl_sync(0xffffffffu, my_off, kk);
+            if (off >= 0) {
+                const RowT *kr, *vr;
+                if (VIRT) {
+                    const int64_t o = off & ~(int64_t(1) << 62);
+                    const bool cur = (off >> 62) != 0;
+                    kr = reinterpret_cast<const RowT *>(cur ? kcur : kc) + o;
+                    vr = reinterpret_cast<const RowT *>(cur ? vcur : vc) + o;
+                } else {
+                    kr = reinterpret_cast<const RowT *>(kw) + off;
+                    vr = reinterpret_cast<const RowT *>(vw) + off;
+                }
+                rkl[kk].ld(kr + PD * lane);
+                rkh[kk].ld(kr + D / 2 + PD * lane);
+                rvl[kk].ld(vr + PD * lane);
+                rvh[kk].ld(vr + D / 2 + PD * lane);
+            }
+        }
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        const int64_t p0 = pi + nb * KB;
+        float klo[KB][PD], khi[KB][PD], vlo[KB][PD], vhi[KB][PD];
+#pragma unroll
+        for (int kk = 0; kk < KB; ++kk) {
+            const int64_t p = p0 + kk;
+            if (p < kend) {
+                rkl[nb * KB + kk].get(klo[kk]);
+                rkh[nb * KB + kk].get(khi[kk]);
+                rvl[nb * KB + kk].get(vlo[kk]);
+                rvh[nb * KB + kk].get(vhi[kk]);
+                if (VIRT) {   // rotate the key pair at window position p
+                    const float2 *cs = a.tab + p * (D / 2) + PD * lane;
+#pragma unroll
+                    for (int e = 0; e < PD; ++e) {
+                        const float2 t = __ldg(cs + e);
+                        const float x0 = klo[kk][e], x1 = khi[kk][e];
+                        klo[kk][e] = x0 * t.x - x1 * t.y;
+                        khi[kk][e] = x1 * t.x + x0 * t.y;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < PD; ++e) klo[kk][e] = khi[kk][e] = vlo[kk][e] = vhi[kk][e] = 0.f;
+            }
+        }
+        // partial dots part[kk*RP + r] over this lane's pairs
+        float part[32];
+#pragma unroll
+        for (int kk = 0; kk < KB; ++kk)
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                float z = 0.f;
+#pragma unroll
+                for (int e = 0; e < PD; ++e)
+                    z = fmaf(qlo[r][e], klo[kk][e], fmaf(qhi[r][e], khi[kk][e], z));
+                part[kk * RP + r] = z;
+            }
+        // transposed reduction: lane i ends with the full dot of index i
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < o; ++i) {
+                const float send = upper ? part[i] : part[i + o];
+                const float keep = upper ? part[i + o] : part[i];
+                part[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+        const int64_t my_p = p0 + lane / RP;
+        const float x = (my_p < kend && my_p <= my_lim) ? part[0] : -INFINITY;
+        // batch max per row (lanes sharing lane % RP), new running max
+        float bm = x;
+#pragma unroll
+        for (int o = RP; o < 32; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+        const float mn_own = fmaxf(m_own, bm);
+        const float pv = x == -INFINITY ? 0.f : exp2f(x - mn_own);
+        m_own = mn_own;
+        float bs = pv;
+#pragma unroll
+        for (int o = RP; o < 32; o <<= 1) bs += __shfl_xor_sync(0xffffffffu, bs, o);
+#pragma unroll
+        for (int r = 0; r < RP; ++r) {
+            const float mn = fmaxf(mrow[r], __shfl_sync(0xffffffffu, bm, r));
+            const float cf = mn == -INFINITY ? 1.f : exp2f(mrow[r] - mn);
+            mrow[r] = mn;
+            lrow[r] = lrow[r] * cf + __shfl_sync(0xffffffffu, bs, r);
+#pragma unroll
+            for (int e = 0; e < PD; ++e) {
+                alo[r][e] *= cf;
+                ahi[r][e] *= cf;
+            }
+        }
+#pragma unroll
+        for (int kk = 0; kk < KB; ++kk)
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                const float pr = __shfl_sync(0xffffffffu, pv, kk * RP + r);
+#pragma unroll
+                for (int e = 0; e < PD; ++e) {
+                    alo[r][e] = fmaf(pr, vlo[kk][e], alo[r][e]);
+                    ahi[r][e] = fmaf(pr, vhi[kk][e], ahi[r][e]);
+                }
+            }
+    }
+    }
+
+    // merge the warps of the CTA
+#pragma unroll
+    for (int r = 0; r < RP; ++r) {
+        if (lane == 0) {
+            s_m[warp][r] = mrow[r];
+            s_l[warp][r] = lrow[r];
+        }
+#pragma unroll
+        for (int e = 0; e < PD; ++e) {
+            s_acc[warp][r][PD * lane + e] = alo[r][e];
+            s_acc[warp][r][D / 2 + PD * lane + e] = ahi[r][e];
+        }
+    }
+    __syncthreads();
+    if (tid < RP) {
+        float mx = -INFINITY;
+        for (int w2 = 0; w2 < kDecWarps; ++w2) mx = fmaxf(mx, s_m[w2][tid]);
+        float l = 0.f;
+        for (int w2 = 0; w2 < kDecWarps; ++w2) {
+            const float wt = s_m[w2][tid] == -INFINITY ? 0.f : exp2f(s_m[w2][tid] - mx);
+            s_m[w2][tid] = wt;   // now a weight
+            l += wt * s_l[w2][tid];
+        }
+        f_m[tid] = mx;
+        f_l[tid] = l;
+    }
+    __syncthreads();
+    for (int x = tid; x < RP * D; x += kDecWarps * 32) {
+        const int r = x / D, i = x % D;
+        float z = 0.f;
+        for (int w2 = 0; w2 < kDecWarps; ++w2) z = fmaf(s_m[w2][r], s_acc[w2][r][i], z);
+        s_acc[0][r][i] = z;   // row r of warp 0's slot is only read by this thread
+    }
+    __syncthreads();
+    split_finish<D, RP>(geo, a, bh, 0, split, nrows, f_m, f_l, &s_acc[0][0][0], &s_acc[1][0][0],
+                        &is_last);
+}
+
+// ---------------------------------------------------------------- staged decode attention
+// The fused step's decode path.  One producer thread walks the CTA's key range
+// of the virtual window in chunks that are contiguous in memory (<= 32 rows,
+// never crossing the end of the global part, of a chosen span, of the local
+// part) and bulk-copies each chunk's K and V rows into a shared-memory ring
+// (cp.async.bulk, mbarrier completion).  Consumer warp w takes chunks w,
+// w+NCW, ... (fixed stage -> warp map, so parity waits never run ahead) and
+// computes as the register kernel above, reading its pair words from shared
+// memory.  RoPE cos/sin come from the fp32 reduced angle at the start of each
+// sub-batch, advanced key by key with the constant one-position rotation.
+constexpr int kTmaCW = 16;                 // consumer warps
+constexpr int kTmaStages = 16;             // multiple of kTmaCW
+
+template <typename T, int D>
+struct TmaShape {
+    static constexpr int kRowBytes = D * Elem<T>::kBytes;
+    static constexpr int kChunk = kRowBytes >= 512 ? 8 : 16;          // rows per ring stage
+    static constexpr int kStageBytes = 2 * kChunk * kRowBytes;         // K rows then V rows
+    static constexpr size_t kRing = size_t(kTmaStages) * kStageBytes;
+};
+static_assert(kTmaStages % kTmaCW == 0, "stage -> warp map must be fixed");
+
+// Chunk of window rows starting at p: its length (contiguous source run).
+__device__ __forceinline__ int chunk_len(const Geom &geo, const WinMap &m, int64_t p, int64_t kend,
+                                         int chunk)
+{
+    const int64_t g_end = m.g_end, nsel = m.nsel_rows, nloc = m.n_loc;
+    int64_t end;
+    if (p < g_end) {
+        end = g_end;
+    } else if (p < g_end + nsel) {
+        const int64_t j = (p - g_end) / geo.S;
+        end = g_end + (j + 1) * geo.S;
+        if (end > g_end + nsel) end = g_end + nsel;
+    } else if (p < g_end + nsel + nloc) {
+        end = g_end + nsel + nloc;
+    } else {
+        end = m.W;
+    }
+    if (end > kend) end = kend;
+    if (end > p + chunk) end = p + chunk;
+    return int(end - p);
+}
+
+template <typename T, int D, int RP>
+__global__ void __launch_bounds__((kTmaCW + 1) * 32, 1)
+attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__restrict__ vc,
+                     const T *__restrict__ kcur, const T *__restrict__ vcur, void *ws)
+{
+    using Sh = TmaShape<T, D>;
+    constexpr int PD = D / 64;            // RoPE pairs per lane
+    constexpr int KB = 32 / RP;           // keys per reduction batch
+    constexpr int RB = Sh::kRowBytes;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint8_t *ring = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Sh::kRing);
+    uint64_t *empty = full + kTmaStages;
+    float *s_acc = reinterpret_cast<float *>(empty + kTmaStages);      // [kTmaCW][RP][D]
+    float *s_m = s_acc + kTmaCW * RP * D;                               // [kTmaCW][RP]
+    float *s_l = s_m + kTmaCW * RP;
+    __shared__ float f_m[RP], f_l[RP];
+    __shared__ float2 freq[D / 2];
+    __shared__ int is_last, abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int split = blockIdx.x;
+    const int64_t bh = blockIdx.z;
+    const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv);
+    const int nrows = geo.g * geo.C;
+    const int32_t *sel_bh = a.sel + bh * geo.k;
+    const WinMap m = make_winmap(geo, sel_bh);
+    const int64_t W = m.W, qpos0 = W - geo.C;
+    int64_t kbeg, kend;
+    split_range(geo, W, a.nsplit, split, 0, nrows, Sh::kChunk, kbeg, kend);
+
+    if (tid == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < kTmaStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init_fence();
+    }
+    if (tid < D / 2) freq[tid] = make_float2(geo.rope_hi[tid], geo.rope_lo[tid]);
+    __syncthreads();
+
+    if (warp == kTmaCW) {
+        // ------------------------------------------------ producer (one thread)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool wrapped = false;
+            for (int64_t p = kbeg; p < kend;) {
+                const int n = chunk_len(geo, m, p, kend, Sh::kChunk);
+                if (wrapped && (*(volatile int *)&abort_flag ||
+                                !mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs))) {
+                    report_status(ws, REATT_ETIMEOUT);
+                    *(volatile int *)&abort_flag = 1;
+                    break;
+                }
+                const int64_t off = win_row_offset(geo, m, sel_bh, bh, int(p), D);
+                const bool cur = (off >> 62) != 0;
+                const int64_t o = off & ~(int64_t(1) << 62);
+                const uint32_t bytes = uint32_t(n) * RB;
+                uint8_t *dst = ring + stage * Sh::kStageBytes;
+                mbar_arrive_expect_tx(&full[stage], 2 * bytes);
+                bulk_load_plain(dst, (cur ? kcur : kc) + o, bytes, &full[stage]);
+                bulk_load_plain(dst + Sh::kChunk * RB, (cur ? vcur : vc) + o, bytes, &full[stage]);
+                p += n;
+                if (++stage == kTmaStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                    wrapped = true;
+                }
+            }
+            for (int k2 = 0; k2 < kTmaStages; ++k2) {   // drain the copies in flight
+                if (--stage < 0) {
+                    stage = kTmaStages - 1;
+                    if (!wrapped) break;
+                    phase ^= 1u;
+                }
+                if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs))
+                    report_status(ws, REATT_ETIMEOUT);
+            }
+        }
+    } else {
+        // ---------------------------------------------------- consumers
+        float qlo[RP][PD], qhi[RP][PD];
+        float2 step[PD];   // (cos, sin) of one position step, per pair
+#pragma unroll
+        for (int e = 0; e < PD; ++e) {
+            const int i = PD * lane + e;
+            rope_cs(1, freq[i].x, freq[i].y, step[e].x, step[e].y);
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                qlo[r][e] = qhi[r][e] = 0.f;
+                if (r < nrows) query_pair<T, D>(geo, freq, a.q, b, h, r, qpos0, i, qlo[r][e], qhi[r][e]);
+            }
+        }
+        const int my_r = lane % RP;
+        const int64_t my_lim = my_r < nrows ? qpos0 + my_r % geo.C : -1;
+        float mrow[RP], lrow[RP], alo[RP][PD], ahi[RP][PD];
+#pragma unroll
+        for (int r = 0; r < RP; ++r) {
+            mrow[r] = -INFINITY;
+            lrow[r] = 0.f;
+#pragma unroll
+            for (int e = 0; e < PD; ++e) alo[r][e] = ahi[r][e] = 0.f;
+        }
+        float m_own = -INFINITY;
+
+        int stage = 0, ci = 0;
+        uint32_t phase = 0;
+        for (int64_t p = kbeg; p < kend; ++ci) {
+            const int n = chunk_len(geo, m, p, kend, Sh::kChunk);
+            const int64_t pc = p;
+            const int st_now = stage;
+            const uint32_t par = phase;
+            p += n;
+            if (++stage == kTmaStages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+            if ((st_now % kTmaCW) != warp) continue;
+            if (__any_sync(0xffffffffu, *(volatile int *)&abort_flag != 0)) continue;
+            const bool ok = mbar_wait_bounded(&full[st_now], par, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) {
+                    report_status(ws, REATT_ETIMEOUT);
+                    *(volatile int *)&abort_flag = 1;
+                }
+                continue;
+            }
+            const uint8_t *kb = ring + st_now * Sh::kStageBytes;
+            const uint8_t *vb = kb + Sh::kChunk * RB;
+            for (int sb = 0; sb < n; sb += KB) {
+                // anchor cos/sin at the first key of the sub-batch
+                float2 cs[PD];
+#pragma unroll
+                for (int e = 0; e < PD; ++e) {
+                    const int i = PD * lane + e;
+                    rope_cs(pc + sb, freq[i].x, freq[i].y, cs[e].x, cs[e].y);
+                }
+                constexpr int EB = Elem<T>::kBytes;
+                float part[32];
+#pragma unroll
+                for (int kk = 0; kk < KB; ++kk) {
+                    const int row = sb + kk;
+                    float klo[PD], khi[PD];
+                    if (row < n) {
+                        PairRaw<T, PD> w0, w1;
+                        w0.lds(kb + row * RB + PD * lane * EB);
+                        w1.lds(kb + row * RB + (D / 2 + PD * lane) * EB);
+                        w0.get(klo);
+                        w1.get(khi);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < PD; ++e) klo[e] = khi[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < PD; ++e) {
+                        const float x0 = klo[e], x1 = khi[e];
+                        klo[e] = x0 * cs[e].x - x1 * cs[e].y;
+                        khi[e] = x1 * cs[e].x + x0 * cs[e].y;
+                        const float c2 = cs[e].x * step[e].x - cs[e].y * step[e].y;
+                        cs[e].y = cs[e].y * step[e].x + cs[e].x * step[e].y;
+                        cs[e].x = c2;
+                    }
+#pragma unroll
+                    for (int r = 0; r < RP; ++r) {
+                        float z = 0.f;
+#pragma unroll
+                        for (int e = 0; e < PD; ++e)
+                            z = fmaf(qlo[r][e], klo[e], fmaf(qhi[r][e], khi[e], z));
+                        part[kk * RP + r] = z;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+                    const bool upper = (lane & o) != 0;
+#pragma unroll
+                    for (int i = 0; i < o; ++i) {
+                        const float send = upper ? part[i] : part[i + o];
+                        const float keep = upper ? part[i + o] : part[i];
+                        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                    }
+                }
+                const int my_row = sb + lane / RP;
+                const int64_t my_p = pc + my_row;
+                const float x = (my_row < n && my_p <= my_lim) ? part[0] : -INFINITY;
+                float bm = x;
+#pragma unroll
+                for (int o = RP; o < 32; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+                const float mn_own = fmaxf(m_own, bm);
+                const float pv = x == -INFINITY ? 0.f : exp2f(x - mn_own);
+                m_own = mn_own;
+                float bs = pv;
+#pragma unroll
+                for (int o = RP; o < 32; o <<= 1) bs += __shfl_xor_sync(0xffffffffu, bs, o);
+#pragma unroll
+                for (int r = 0; r < RP; ++r) {
+                    const float mn = fmaxf(mrow[r], __shfl_sync(0xffffffffu, bm, r));
+                    const float cf = mn == -INFINITY ? 1.f : exp2f(mrow[r] - mn);
+                    mrow[r] = mn;
+                    lrow[r] = lrow[r] * cf + __shfl_sync(0xffffffffu, bs, r);
+#pragma unroll
+                    for (int e = 0; e < PD; ++e) {
+                        alo[r][e] *= cf;
+                        ahi[r][e] *= cf;
+                    }
+                }
+#pragma unroll
+                for (int kk = 0; kk < KB; ++kk) {
+                    const int row = sb + kk;
+                    float vlo[PD], vhi[PD];
+                    if (row < n) {
+                        PairRaw<T, PD> w2, w3;
+                        w2.lds(vb + row * RB + PD * lane * EB);
+                        w3.lds(vb + row * RB + (D / 2 + PD * lane) * EB);
+                        w2.get(vlo);
+                        w3.get(vhi);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < PD; ++e) vlo[e] = vhi[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int r = 0; r < RP; ++r) {
+                        const float pr = __shfl_sync(0xffffffffu, pv, kk * RP + r);
+#pragma unroll
+                        for (int e = 0; e < PD; ++e) {
+                            alo[r][e] = fmaf(pr, vlo[e], alo[r][e]);
+                            ahi[r][e] = fmaf(pr, vhi[e], ahi[r][e]);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st_now]);   // chunk consumed: hand the stage back
+        }
+        // this warp's state to shared memory
+#pragma unroll
+        for (int r = 0; r < RP; ++r) {
+            if (lane == 0) {
+                s_m[warp * RP + r] = mrow[r];
+                s_l[warp * RP + r] = lrow[r];
+            }
+#pragma unroll
+            for (int e = 0; e < PD; ++e) {
+                s_acc[(warp * RP + r) * D + PD * lane + e] = alo[r][e];
+                s_acc[(warp * RP + r) * D + D / 2 + PD * lane + e] = ahi[r][e];
+            }
+        }
+    }
+    __syncthreads();
+    // merge the consumer warps
+    if (tid < RP) {
+        float mx = -INFINITY;
+        for (int w2 = 0; w2 < kTmaCW; ++w2) mx = fmaxf(mx, s_m[w2 * RP + tid]);
+        float l = 0.f;
+        for (int w2 = 0; w2 < kTmaCW; ++w2) {
+            const float mv = s_m[w2 * RP + tid];
+            const float wt = mv == -INFINITY ? 0.f : exp2f(mv - mx);
+            s_m[w2 * RP + tid] = wt;
+            l += wt * s_l[w2 * RP + tid];
+        }
+        f_m[tid] = mx;
+        f_l[tid] = l;
+    }
+    __syncthreads();
+    for (int x = tid; x < RP * D; x += blockDim.x) {
+        const int r = x / D, i = x % D;
+        float z = 0.f;
+        for (int w2 = 0; w2 < kTmaCW; ++w2) z = fmaf(s_m[w2 * RP + r], s_acc[(w2 * RP + r) * D + i], z);
+        s_acc[r * D + i] = z;   // slot (warp 0, r): only this thread touches element i
+    }
+    __syncthreads();
+    split_finish<D, RP>(geo, a, bh, 0, split, nrows, f_m, f_l, s_acc, s_acc + RP * D, &is_last);
+}
+
+template <typename T, int D>
+cudaError_t launch_staged_attn(const Geom &geo, const AttnArgs &a, int RP, const void *kc,
+                               const void *vc, const void *kcur, const void *vcur, void *ws,
+                               cudaStream_t st)
+{
+    using Sh = TmaShape<T, D>;
+    dim3 grid(unsigned(a.nsplit), 1u, unsigned(geo.B * geo.Hkv));
+    const T *k = static_cast<const T *>(kc), *v = static_cast<const T *>(vc);
+    const T *kq = static_cast<const T *>(kcur), *vq = static_cast<const T *>(vcur);
+#define REATT_STAGED(RPV)                                                                      \
+    do {                                                                                       \
+        const size_t smem = Sh::kRing + 2 * kTmaStages * sizeof(uint64_t) +                   \
+                            size_t(kTmaCW) * RPV * (D + 2) * sizeof(float);                    \
+        auto kern = attend_staged_kernel<T, D, RPV>;                                           \
+        cudaError_t e =                                                                        \
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)); \
+        if (e != cudaSuccess) return e;                                                        \
+        kern<<<grid, (kTmaCW + 1) * 32, smem, st>>>(geo, a, k, v, kq, vq, ws);                 \
+    } while (0)
+    switch (RP) {
+    case 1: REATT_STAGED(1); break;
+    case 2: REATT_STAGED(2); break;
+    case 4: REATT_STAGED(4); break;
+    default: REATT_STAGED(8); break;
+    }
+#undef REATT_STAGED
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- tile attention
+// Many query rows per KV head (chunked prefill): a CTA owns QB rows and stages
+// key/value tiles of 64 rows through shared memory (rotated on the way in when
+// read from the un-rotated cache), with register prefetch of the next tile.
+template <int D, int QB>
+struct AttnSmem {
+    static constexpr int kKS = D + 4;                     // padded key row (floats)
+    static constexpr size_t kQ = size_t(QB) * D * 4;
+    static constexpr size_t kK = size_t(kKT) * kKS * 4;
+    static constexpr size_t kV = size_t(kKT) * D * 4;
+    static constexpr size_t kP = size_t(QB) * kKT * 4;
+    static constexpr size_t kRow = size_t(QB) * 4 * 4;   // m, l, corr, spare
+    static constexpr size_t kTotal = kQ + kK + kV + kP + kRow;
+};
+
+// Raw (unconverted) 16-byte vectors of one half-row item of K and V.
+struct RawKV {
+    uint4 klo, khi, vlo, vhi;
+};
+
 template <typename T, int D, bool VIRT>
 struct KvSource;
 
-// Virtual window: rows straight from the un-rotated cache / current tokens.
+// Virtual window: rows straight from the un-rotated cache / current tokens,
+// rotated with the per-step cos/sin table.
 template <typename T, int D>
 struct KvSource<T, D, true> {
     const T *kc, *vc, *kcur, *vcur;
-    const int32_t *sel;
+    const float2 *tab;
     static constexpr int V = Elem<T>::kVec;
-    __device__ __forceinline__ void load(const Geom &geo, const WinMap &m, int64_t bh,
-                                         const int32_t *sel_bh, int64_t p, int v,
-                                         const double *ifreq, float (&klo)[V], float (&khi)[V],
-                                         float (&vlo)[V], float (&vhi)[V]) const
+    __device__ __forceinline__ RawKV fetch(const Geom &geo, const WinMap &m, int64_t bh,
+                                           const int32_t *sel_bh, int64_t p, int v) const
     {
         const int64_t s = win_src(geo, m, sel_bh, p);
         const T *kr, *vr;
@@ -162,17 +955,29 @@ struct KvSource<T, D, true> {
             kr = kcur + (bh * geo.C + (-s - 1)) * D;
             vr = vcur + (bh * geo.C + (-s - 1)) * D;
         }
+        RawKV r;
+        r.klo = ldg_stream(kr + v * V);
+        r.khi = ldg_stream(kr + D / 2 + v * V);
+        r.vlo = ldg_stream(vr + v * V);
+        r.vhi = ldg_stream(vr + D / 2 + v * V);
+        return r;
+    }
+    __device__ __forceinline__ void finish(const RawKV &r, int64_t p, int v, float (&klo)[V],
+                                           float (&khi)[V], float (&vlo)[V], float (&vhi)[V]) const
+    {
         float a[V], b[V];
-        Elem<T>::unpack(ldg_stream(kr + v * V), a);
-        Elem<T>::unpack(ldg_stream(kr + D / 2 + v * V), b);
-        Elem<T>::unpack(ldg_stream(vr + v * V), vlo);
-        Elem<T>::unpack(ldg_stream(vr + D / 2 + v * V), vhi);
+        Elem<T>::unpack(r.klo, a);
+        Elem<T>::unpack(r.khi, b);
+        Elem<T>::unpack(r.vlo, vlo);
+        Elem<T>::unpack(r.vhi, vhi);
+        const float4 *cs = reinterpret_cast<const float4 *>(tab + p * (D / 2) + v * V);
 #pragma unroll
-        for (int e = 0; e < V; ++e) {
-            float c, sn;
-            rope_cs(p, ifreq[v * V + e], c, sn);
-            klo[e] = a[e] * c - b[e] * sn;
-            khi[e] = b[e] * c + a[e] * sn;
+        for (int e = 0; e < V; e += 2) {
+            const float4 t = __ldg(cs + e / 2);   // (cos, sin) of elements e, e+1
+            klo[e] = a[e] * t.x - b[e] * t.y;
+            khi[e] = b[e] * t.x + a[e] * t.y;
+            klo[e + 1] = a[e + 1] * t.z - b[e + 1] * t.w;
+            khi[e + 1] = b[e + 1] * t.z + a[e + 1] * t.w;
         }
     }
 };
@@ -182,40 +987,42 @@ template <typename T, int D>
 struct KvSource<T, D, false> {
     const float *kw, *vw;
     static constexpr int V = 4;
-    __device__ __forceinline__ void load(const Geom &geo, const WinMap &, int64_t bh,
-                                         const int32_t *, int64_t p, int v, const double *,
-                                         float (&klo)[V], float (&khi)[V], float (&vlo)[V],
-                                         float (&vhi)[V]) const
+    __device__ __forceinline__ RawKV fetch(const Geom &geo, const WinMap &, int64_t bh,
+                                           const int32_t *, int64_t p, int v) const
     {
         const float *kr = kw + (bh * geo.Wmax + p) * D;
         const float *vr = vw + (bh * geo.Wmax + p) * D;
-        Elem<float>::unpack(ldg_stream(kr + v * V), klo);
-        Elem<float>::unpack(ldg_stream(kr + D / 2 + v * V), khi);
-        Elem<float>::unpack(ldg_stream(vr + v * V), vlo);
-        Elem<float>::unpack(ldg_stream(vr + D / 2 + v * V), vhi);
+        RawKV r;
+        r.klo = ldg_stream(kr + v * V);
+        r.khi = ldg_stream(kr + D / 2 + v * V);
+        r.vlo = ldg_stream(vr + v * V);
+        r.vhi = ldg_stream(vr + D / 2 + v * V);
+        return r;
     }
-};
-
-struct AttnArgs {
-    const void *q;
-    const int32_t *sel;       // virtual window
-    const int32_t *win_len;   // materialised window
-    float *out;
-    float *part;              // [BH][nqb][nsplit][QB][D+2]
-    uint32_t *ticket;         // [BH][nqb]
-    int nqb, nsplit;
+    __device__ __forceinline__ void finish(const RawKV &r, int64_t, int, float (&klo)[V],
+                                           float (&khi)[V], float (&vlo)[V], float (&vhi)[V]) const
+    {
+        Elem<float>::unpack(r.klo, klo);
+        Elem<float>::unpack(r.khi, khi);
+        Elem<float>::unpack(r.vlo, vlo);
+        Elem<float>::unpack(r.vhi, vhi);
+    }
 };
 
 template <typename T, int D, int QB, bool VIRT>
 __global__ void __launch_bounds__(kAttnThreads)
-attend_kernel(Geom geo, AttnArgs a, KvSource<T, D, VIRT> src)
+attend_tile_kernel(Geom geo, AttnArgs a, KvSource<T, D, VIRT> src)
 {
     using Sm = AttnSmem<D, QB>;
     constexpr int V = KvSource<T, D, VIRT>::V;
-    constexpr int HV = D / 2 / V;
-    constexpr int NACC = QB * D / kAttnThreads;
-    constexpr int NLOG = QB * kKT / kAttnThreads;
-    static_assert(NACC >= 1 && NLOG >= 1, "tile shape");
+    constexpr int HV = D / 2 / V;                          // half-row vectors
+    constexpr int NITEM = kKT * HV / kAttnThreads;         // load items per thread
+    constexpr int NR = QB / 4;                             // logit rows per thread
+    constexpr int D4 = D / 4;
+    constexpr int NACC = (QB * D4 + kAttnThreads - 1) / kAttnThreads;
+    constexpr int KS = Sm::kKS;
+    static_assert(NITEM >= 1 && kKT * HV % kAttnThreads == 0, "tile shape");
+    static_assert(kAttnThreads % kKT == 0 && QB % 4 == 0, "tile shape");
     extern __shared__ __align__(16) uint8_t smem[];
     float *Qs = reinterpret_cast<float *>(smem);
     float *Ks = reinterpret_cast<float *>(smem + Sm::kQ);
@@ -224,10 +1031,12 @@ attend_kernel(Geom geo, AttnArgs a, KvSource<T, D, VIRT> src)
     float *m_run = reinterpret_cast<float *>(smem + Sm::kQ + Sm::kK + Sm::kV + Sm::kP);
     float *l_run = m_run + QB;
     float *corr = l_run + QB;
-    double *ifreq = reinterpret_cast<double *>(smem + Sm::kQ + Sm::kK + Sm::kV + Sm::kP + Sm::kRow);
     __shared__ int is_last;
+    __shared__ float2 freq[D / 2];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid < D / 2) freq[tid] = make_float2(geo.rope_hi[tid], geo.rope_lo[tid]);
+    __syncthreads();
     const int split = blockIdx.x, qb = blockIdx.y;
     const int64_t bh = blockIdx.z;
     const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv);
@@ -236,111 +1045,103 @@ attend_kernel(Geom geo, AttnArgs a, KvSource<T, D, VIRT> src)
     const int nrows = R - r0 < QB ? R - r0 : QB;
 
     const int32_t *sel_bh = VIRT ? a.sel + bh * geo.k : nullptr;
-    WinMap m;
-    if (VIRT) {
-        m = make_winmap(geo, sel_bh);
-    } else {
-        m.g_end = m.loc_begin = m.n_loc = m.nsel_rows = 0;
-        int64_t wl = a.win_len[bh];   // caller data: keep every read inside the window
-        m.W = wl < geo.C ? geo.C : (wl > geo.Wmax ? geo.Wmax : wl);
-    }
+    const WinMap m = attn_winmap(geo, a, VIRT, bh, sel_bh);
     const int64_t W = m.W;
-    const int64_t qpos0 = W - geo.C;                    // position of query c = 0
+    const int64_t qpos0 = W - geo.C;                       // position of query c = 0
+    int64_t kbeg, kend;
+    split_range(geo, W, a.nsplit, split, r0, nrows, kKT, kbeg, kend);
 
-    for (int i = tid; i < D / 2; i += kAttnThreads)
-        ifreq[i] = rope_inv_freq_over_pi(i, D, geo.base);
+    // first tile's loads go out before anything else
+    RawKV raw[NITEM];
+    auto fetch_tile = [&](int64_t t0) {
+#pragma unroll
+        for (int u = 0; u < NITEM; ++u) {
+            const int x = tid + u * kAttnThreads, key = x / HV, v = x % HV;
+            if (t0 + key < kend) raw[u] = src.fetch(geo, m, bh, sel_bh, t0 + key, v);
+        }
+    };
+    if (kbeg < kend) fetch_tile(kbeg);
+
     for (int r = tid; r < QB; r += kAttnThreads) {
         m_run[r] = -INFINITY;
         l_run[r] = 0.f;
     }
-    __syncthreads();
-
-    // rotated, pre-scaled queries: log2(e)/sqrt(d) folds the softmax scale
-    const float qscale = 1.4426950408889634f / sqrtf(float(D));
     for (int x = tid; x < QB * (D / 2); x += kAttnThreads) {
         const int rr = x / (D / 2), i = x % (D / 2);
         float lo = 0.f, hi = 0.f;
-        if (rr < nrows) {
-            const int r = r0 + rr, j = h * geo.g + r / geo.C, c = r % geo.C;
-            const T *qr = static_cast<const T *>(a.q) + ((int64_t(b) * geo.Hq + j) * geo.C + c) * D;
-            const float x0 = Elem<T>::one(qr, i), x1 = Elem<T>::one(qr, i + D / 2);
-            float cs, sn;
-            rope_cs(qpos0 + c, ifreq[i], cs, sn);
-            lo = (x0 * cs - x1 * sn) * qscale;
-            hi = (x1 * cs + x0 * sn) * qscale;
-        }
+        if (rr < nrows) query_pair<T, D>(geo, freq, a.q, b, h, r0 + rr, qpos0, i, lo, hi);
         Qs[rr * D + i] = lo;
         Qs[rr * D + i + D / 2] = hi;
     }
 
-    // key range of this split (multiple of the tile), clipped by causality
-    int64_t chunk = (W + a.nsplit - 1) / a.nsplit;
-    chunk = (chunk + kKT - 1) / kKT * kKT;
-    const int64_t kbeg = int64_t(split) * chunk;
-    int64_t kend = kbeg + chunk;
-    if (kend > W) kend = W;
-    const int last_row = r0 + nrows - 1;
-    const int c_max = (last_row / geo.C == r0 / geo.C) ? last_row % geo.C : geo.C - 1;
-    if (kend > qpos0 + c_max + 1) kend = qpos0 + c_max + 1;
-
-    float acc[NACC];
+    float4 acc[NACC];
 #pragma unroll
-    for (int u = 0; u < NACC; ++u) acc[u] = 0.f;
+    for (int u = 0; u < NACC; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
 
     for (int64_t t0 = kbeg; t0 < kend; t0 += kKT) {
         const int nk = int(kend - t0 < kKT ? kend - t0 : kKT);
-        __syncthreads();
-        for (int x = tid; x < kKT * HV; x += kAttnThreads) {
-            const int key = x / HV, v = x % HV;
+        __syncthreads();   // previous tile fully consumed
+#pragma unroll
+        for (int u = 0; u < NITEM; ++u) {
+            const int x = tid + u * kAttnThreads, key = x / HV, v = x % HV;
             float klo[V], khi[V], vlo[V], vhi[V];
             if (key < nk) {
-                src.load(geo, m, bh, sel_bh, t0 + key, v, ifreq, klo, khi, vlo, vhi);
+                src.finish(raw[u], t0 + key, v, klo, khi, vlo, vhi);
             } else {
 #pragma unroll
                 for (int e = 0; e < V; ++e) klo[e] = khi[e] = vlo[e] = vhi[e] = 0.f;
             }
 #pragma unroll
-            for (int e = 0; e < V; ++e) {
+            for (int e = 0; e < V; e += 4) {
                 const int i = v * V + e;
-                Ks[key * (D + 1) + i] = klo[e];
-                Ks[key * (D + 1) + i + D / 2] = khi[e];
-                Vs[key * D + i] = vlo[e];
-                Vs[key * D + i + D / 2] = vhi[e];
+                *reinterpret_cast<float4 *>(Ks + key * KS + i) =
+                    make_float4(klo[e], klo[e + 1], klo[e + 2], klo[e + 3]);
+                *reinterpret_cast<float4 *>(Ks + key * KS + i + D / 2) =
+                    make_float4(khi[e], khi[e + 1], khi[e + 2], khi[e + 3]);
+                *reinterpret_cast<float4 *>(Vs + key * D + i) =
+                    make_float4(vlo[e], vlo[e + 1], vlo[e + 2], vlo[e + 3]);
+                *reinterpret_cast<float4 *>(Vs + key * D + i + D / 2) =
+                    make_float4(vhi[e], vhi[e + 1], vhi[e + 2], vhi[e + 3]);
             }
         }
+        if (t0 + kKT < kend) fetch_tile(t0 + kKT);   // next tile in flight during compute
         __syncthreads();
-        // logits (log2 domain), causal mask per row
+
+        // logits (log2 domain) for rows rg, rg+4, ...; causal mask per row
+        {
+            const int key = tid % kKT, rg = tid / kKT;
+            float lg[NR];
 #pragma unroll
-        for (int u = 0; u < NLOG; ++u) {
-            const int x = tid + u * kAttnThreads;
-            const int rr = x / kKT, key = x % kKT;
-            float s = -INFINITY;
-            if (rr < nrows && key < nk) {
-                const int c = (r0 + rr) % geo.C;
-                if (t0 + key <= qpos0 + c) {
-                    const float *qv = Qs + rr * D, *kv = Ks + key * (D + 1);
-                    float z = 0.f;
-#pragma unroll 16
-                    for (int i = 0; i < D; ++i) z = fmaf(qv[i], kv[i], z);
-                    s = z;
+            for (int j = 0; j < NR; ++j) lg[j] = 0.f;
+            const float4 *k4 = reinterpret_cast<const float4 *>(Ks + key * KS);
+#pragma unroll 4
+            for (int d4 = 0; d4 < D4; ++d4) {
+                const float4 kv = k4[d4];
+#pragma unroll
+                for (int j = 0; j < NR; ++j) {
+                    const float4 qv = reinterpret_cast<const float4 *>(Qs + (rg + 4 * j) * D)[d4];
+                    lg[j] = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, lg[j]))));
                 }
             }
-            Ps[rr * kKT + key] = s;
+#pragma unroll
+            for (int j = 0; j < NR; ++j) {
+                const int rr = rg + 4 * j;
+                const int c = (r0 + rr) % geo.C;
+                const bool ok = rr < nrows && key < nk && t0 + key <= qpos0 + c;
+                Ps[rr * kKT + key] = ok ? lg[j] : -INFINITY;
+            }
         }
         __syncthreads();
         // online softmax, one warp per row
         for (int rr = warp; rr < nrows; rr += kAttnThreads / 32) {
-            float v0 = Ps[rr * kKT + lane], v1 = Ps[rr * kKT + lane + 32];
+            const float v0 = Ps[rr * kKT + lane], v1 = Ps[rr * kKT + lane + 32];
             float mx = fmaxf(v0, v1);
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             const float m_old = m_run[rr];
             const float m_new = fmaxf(m_old, mx);
-            float cf, p0, p1;
-            if (m_new == -INFINITY) {
-                cf = 1.f;
-                p0 = p1 = 0.f;
-            } else {
+            float cf = 1.f, p0 = 0.f, p1 = 0.f;
+            if (m_new != -INFINITY) {
                 cf = exp2f(m_old - m_new);
                 p0 = exp2f(v0 - m_new);
                 p1 = exp2f(v1 - m_new);
@@ -350,7 +1151,6 @@ attend_kernel(Geom geo, AttnArgs a, KvSource<T, D, VIRT> src)
             float sum = p0 + p1;
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            __syncwarp();
             if (lane == 0) {
                 m_run[rr] = m_new;
                 l_run[rr] = l_run[rr] * cf + sum;
@@ -358,84 +1158,46 @@ attend_kernel(Geom geo, AttnArgs a, KvSource<T, D, VIRT> src)
             }
         }
         __syncthreads();
-        // acc = acc * corr + P V
+        // acc = acc * corr + P V, one (row, 4 dims) item per slot
 #pragma unroll
         for (int u = 0; u < NACC; ++u) {
             const int x = tid + u * kAttnThreads;
-            const int rr = x / D, i = x % D;
-            if (rr < nrows) {
-                float z = acc[u] * corr[rr];
+            const int rr = x / D4, d4 = x % D4;
+            if (x < QB * D4 && rr < nrows) {
+                const float cf = corr[rr];
+                float4 z = make_float4(acc[u].x * cf, acc[u].y * cf, acc[u].z * cf, acc[u].w * cf);
                 const float *pr = Ps + rr * kKT;
+                const float4 *v4 = reinterpret_cast<const float4 *>(Vs) + d4;
 #pragma unroll 8
-                for (int key = 0; key < nk; ++key) z = fmaf(pr[key], Vs[key * D + i], z);
+                for (int key = 0; key < nk; ++key) {
+                    const float p = pr[key];
+                    const float4 vv = v4[key * D4];
+                    z.x = fmaf(p, vv.x, z.x);
+                    z.y = fmaf(p, vv.y, z.y);
+                    z.z = fmaf(p, vv.z, z.z);
+                    z.w = fmaf(p, vv.w, z.w);
+                }
                 acc[u] = z;
             }
         }
     }
     __syncthreads();
-
-    if (a.nsplit == 1) {
-#pragma unroll
-        for (int u = 0; u < NACC; ++u) {
-            const int x = tid + u * kAttnThreads;
-            const int rr = x / D, i = x % D;
-            if (rr < nrows) {
-                const int r = r0 + rr, j = h * geo.g + r / geo.C, c = r % geo.C;
-                a.out[((int64_t(b) * geo.Hq + j) * geo.C + c) * D + i] = acc[u] / l_run[rr];
-            }
-        }
-        return;
-    }
-
-    // partials of this split, then the last CTA of (bh, qb) combines
-    const int64_t pbase = (bh * a.nqb + qb) * a.nsplit;
-    float *mine = a.part + (pbase + split) * int64_t(QB) * (D + 2);
+    // accumulators to shared memory (the Q tile is free now), then finish
 #pragma unroll
     for (int u = 0; u < NACC; ++u) {
         const int x = tid + u * kAttnThreads;
-        const int rr = x / D, i = x % D;
-        if (rr < nrows) mine[rr * (D + 2) + 2 + i] = acc[u];
-    }
-    for (int rr = tid; rr < nrows; rr += kAttnThreads) {
-        mine[rr * (D + 2)] = m_run[rr];
-        mine[rr * (D + 2) + 1] = l_run[rr];
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const uint32_t prev = atomicAdd(&a.ticket[bh * a.nqb + qb], 1u);
-        is_last = prev == uint32_t(a.nsplit - 1);
+        if (x < QB * D4) reinterpret_cast<float4 *>(Qs)[x] = acc[u];
     }
     __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    const float *all = a.part + pbase * int64_t(QB) * (D + 2);
-    for (int x = tid; x < nrows * D; x += kAttnThreads) {
-        const int rr = x / D, i = x % D;
-        float mx = -INFINITY;
-        for (int s = 0; s < a.nsplit; ++s)
-            mx = fmaxf(mx, __ldcg(all + (int64_t(s) * QB + rr) * (D + 2)));
-        float den = 0.f, num = 0.f;
-        for (int s = 0; s < a.nsplit; ++s) {
-            const float *ps = all + (int64_t(s) * QB + rr) * (D + 2);
-            const float ms = __ldcg(ps);
-            if (ms == -INFINITY) continue;
-            const float w = exp2f(ms - mx);
-            den += w * __ldcg(ps + 1);
-            num += w * __ldcg(ps + 2 + i);
-        }
-        const int r = r0 + rr, j = h * geo.g + r / geo.C, c = r % geo.C;
-        a.out[((int64_t(b) * geo.Hq + j) * geo.C + c) * D + i] = num / den;
-    }
-    if (tid == 0) a.ticket[bh * a.nqb + qb] = 0u;   // ready for the next call
+    split_finish<D, QB>(geo, a, bh, qb, split, nrows, m_run, l_run, Qs, Ks, &is_last);
 }
 
 template <typename T, int D, int QB, bool VIRT>
-cudaError_t launch_attn(const Geom &geo, const AttnArgs &a, const KvSource<T, D, VIRT> &src,
+cudaError_t launch_tile(const Geom &geo, const AttnArgs &a, const KvSource<T, D, VIRT> &src,
                         cudaStream_t st)
 {
     using Sm = AttnSmem<D, QB>;
-    auto kern = attend_kernel<T, D, QB, VIRT>;
+    auto kern = attend_tile_kernel<T, D, QB, VIRT>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Sm::kTotal));
     if (e != cudaSuccess) return e;
@@ -445,11 +1207,24 @@ cudaError_t launch_attn(const Geom &geo, const AttnArgs &a, const KvSource<T, D,
 }
 
 template <typename T, int D, bool VIRT>
-cudaError_t dispatch_qb(const Geom &geo, const AttnArgs &a, const KvSource<T, D, VIRT> &src,
-                        int QB, cudaStream_t st)
+cudaError_t launch_decode_attn(const Geom &geo, const AttnArgs &a, int RP, const void *kc,
+                               const void *vc, const void *kcur, const void *vcur,
+                               const float *kw, const float *vw, cudaStream_t st)
 {
-    if (QB == 8) return launch_attn<T, D, 8, VIRT>(geo, a, src, st);
-    return launch_attn<T, D, 64, VIRT>(geo, a, src, st);
+    dim3 grid(unsigned(a.nsplit), 1u, unsigned(geo.B * geo.Hkv));
+    const T *k = static_cast<const T *>(kc), *v = static_cast<const T *>(vc);
+    const T *kq = static_cast<const T *>(kcur), *vq = static_cast<const T *>(vcur);
+#define REATT_DEC(RPV)                                                                         \
+    attend_decode_kernel<T, D, RPV, VIRT><<<grid, kDecWarps * 32, 0, st>>>(geo, a, k, v, kq,   \
+                                                                            vq, kw, vw)
+    switch (RP) {
+    case 1: REATT_DEC(1); break;
+    case 2: REATT_DEC(2); break;
+    case 4: REATT_DEC(4); break;
+    default: REATT_DEC(8); break;
+    }
+#undef REATT_DEC
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -458,25 +1233,52 @@ AttnPlan attn_plan(const Geom &geo)
 {
     AttnPlan p;
     const int64_t R = int64_t(geo.g) * geo.C;
-    p.QB = R <= 8 ? 8 : 64;
+    const int64_t BH = int64_t(geo.B) * geo.Hkv;
+    if (R <= 8) {   // warp kernel: one query block of RP rows
+        p.decode = true;
+        p.QB = R <= 1 ? 1 : R <= 2 ? 2 : R <= 4 ? 4 : 8;
+        p.nqb = 1;
+        int64_t ns = (kDecodeCtas + BH - 1) / BH;
+        const int64_t max_split = (geo.Wmax + kMinSplitKeys - 1) / kMinSplitKeys;
+        const int64_t cap = int64_t(kDecWarps - 1) * geo.d;   // combine scratch (floats / QB)
+        if (ns > max_split) ns = max_split;
+        if (ns > cap) ns = cap;
+        p.nsplit = int(ns < 1 ? 1 : ns);
+        return p;
+    }
+    p.decode = false;
+    p.QB = 64;
     p.nqb = int((R + p.QB - 1) / p.QB);
-    const int64_t base = int64_t(geo.B) * geo.Hkv * p.nqb;
-    const int64_t max_split = (geo.Wmax + kKT - 1) / kKT;
+    const int64_t base = BH * p.nqb;
+    // at least kMinSplitKeys keys per split, about kTargetCtas CTAs in all, and
+    // the combine's weights must fit the key tile (nsplit * QB <= kKT * (D+4))
+    int64_t max_split = (geo.Wmax + kMinSplitKeys - 1) / kMinSplitKeys;
+    const int64_t cap = int64_t(kKT) * (geo.d + 4) / p.QB;
+    if (max_split > cap) max_split = cap;
     int64_t ns = 1;
     if (base < kTargetCtas) ns = (kTargetCtas + base - 1) / base;
     if (ns > max_split) ns = max_split;
-    if (ns < 1) ns = 1;
-    p.nsplit = int(ns);
+    p.nsplit = int(ns < 1 ? 1 : ns);
     return p;
 }
 
-size_t attend_ws_bytes(const Geom &geo, size_t *ticket_bytes)
+size_t attend_ws_bytes(const Geom &geo, size_t *ticket_bytes, size_t *ml_off)
 {
     const AttnPlan p = attn_plan(geo);
     const size_t nt = size_t(geo.B) * geo.Hkv * p.nqb;
     *ticket_bytes = (nt * sizeof(uint32_t) + 255) / 256 * 256;
-    if (p.nsplit == 1) return *ticket_bytes;
-    return *ticket_bytes + nt * p.nsplit * p.QB * (geo.d + 2) * sizeof(float);
+    if (p.nsplit == 1) {
+        *ml_off = *ticket_bytes;
+        return *ticket_bytes;
+    }
+    const size_t acc = (nt * p.nsplit * p.QB * geo.d * sizeof(float) + 255) / 256 * 256;
+    *ml_off = *ticket_bytes + acc;
+    return *ticket_bytes + acc + nt * p.nsplit * p.QB * sizeof(float2);
+}
+
+size_t rope_table_bytes(const Geom &geo)
+{
+    return size_t(geo.Wmax) * (geo.d / 2) * sizeof(float2);
 }
 
 cudaError_t launch_gather_rope(const Geom &geo, const void *kc, const void *vc, const void *kcur,
@@ -501,31 +1303,40 @@ cudaError_t launch_gather_rope(const Geom &geo, const void *kc, const void *vc, 
 
 cudaError_t launch_attend(const Geom &geo, const void *q, const float *kw, const float *vw,
                           const int32_t *win_len, const void *kc, const void *vc,
-                          const void *kcur, const void *vcur, const int32_t *sel, float *out,
-                          void *scratch, bool virt, cudaStream_t st)
+                          const void *kcur, const void *vcur, const int32_t *sel,
+                          const float2 *rope_tab, float *out, void *scratch, void *ws, bool virt,
+                          cudaStream_t st)
 {
     const AttnPlan p = attn_plan(geo);
-    size_t tb = 0;
-    attend_ws_bytes(geo, &tb);
+    size_t tb = 0, mo = 0;
+    attend_ws_bytes(geo, &tb, &mo);
     AttnArgs a;
     a.q = q;
     a.sel = sel;
     a.win_len = win_len;
+    a.tab = rope_tab;
     a.out = out;
     a.ticket = static_cast<uint32_t *>(scratch);
-    a.part = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + tb);
+    a.part_acc = reinterpret_cast<float *>(static_cast<uint8_t *>(scratch) + tb);
+    a.part_ml = reinterpret_cast<float2 *>(static_cast<uint8_t *>(scratch) + mo);
     a.nqb = p.nqb;
     a.nsplit = p.nsplit;
 #define REATT_ATT(T, D)                                                                        \
     do {                                                                                       \
+        if (p.decode) {                                                                        \
+            if (virt)                                                                          \
+                return launch_staged_attn<T, D>(geo, a, p.QB, kc, vc, kcur, vcur, ws, st);     \
+            return launch_decode_attn<T, D, false>(geo, a, p.QB, nullptr, nullptr, nullptr,    \
+                                                   nullptr, kw, vw, st);                       \
+        }                                                                                      \
         if (virt) {                                                                            \
             KvSource<T, D, true> s{static_cast<const T *>(kc), static_cast<const T *>(vc),     \
                                    static_cast<const T *>(kcur), static_cast<const T *>(vcur), \
-                                   sel};                                                       \
-            return dispatch_qb<T, D, true>(geo, a, s, p.QB, st);                               \
+                                   rope_tab};                                                  \
+            return launch_tile<T, D, 64, true>(geo, a, s, st);                                 \
         }                                                                                      \
         KvSource<T, D, false> s{kw, vw};                                                       \
-        return dispatch_qb<T, D, false>(geo, a, s, p.QB, st);                                  \
+        return launch_tile<T, D, 64, false>(geo, a, s, st);                                    \
     } while (0)
     if (geo_is_bf16(geo)) {
         if (geo.d == 128) REATT_ATT(uint16_t, 128);

@@ -21,6 +21,10 @@ struct Geom {
     int64_t Wmax;       // G + k*S + L + C
     double base;        // RoPE base
     int dtype;          // reatt_dtype of q, caches, current tokens
+    // RoPE frequency of pair i in half-turns, base^(-2i/d) / pi, computed on
+    // the host in fp64 and split into fp32 hi + lo (hi + lo == value to ~2^-48)
+    float rope_hi[64];
+    float rope_lo[64];
 };
 
 // Workspace header: a status word kept at offset 0 of every workspace.
@@ -90,18 +94,19 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p)
 }
 
 // ----------------------------------------------------------------- RoPE
-// cos/sin of pos * base^(-2i/d).  The angle is formed and reduced modulo 2*pi
-// in fp64 (in units of pi), then evaluated in fp32 by sincospif on [-1, 1].
-__device__ __forceinline__ double rope_inv_freq_over_pi(int i, int d, double base)
+// cos/sin of pos * base^(-2i/d) in fp32 only.  The frequency comes as an
+// unevaluated sum hi + lo (half-turns).  pos*hi is split exactly into its
+// rounded value and the rounding error (fma), the rounded value is reduced
+// modulo 2 exactly (even-integer subtraction of a nearby float), and the small
+// terms are added back, so the reduced argument carries ~1 ulp error on
+// [-1, 1] for positions below 2^24; sincospif then evaluates it.
+__device__ __forceinline__ void rope_cs(int64_t pos, float hi, float lo, float &c, float &s)
 {
-    return pow(base, -2.0 * static_cast<double>(i) / static_cast<double>(d)) *
-           0.31830988618379067154;   // 1/pi
-}
-__device__ __forceinline__ void rope_cs(int64_t pos, double ifreq_over_pi, float &c, float &s)
-{
-    double x = static_cast<double>(pos) * ifreq_over_pi;   // angle / pi
-    x -= 2.0 * rint(0.5 * x);                                // now in [-1, 1]
-    sincospif(static_cast<float>(x), &s, &c);
+    const float p = static_cast<float>(pos);          // exact for pos < 2^24
+    const float ph = p * hi;
+    const float pe = fmaf(p, hi, -ph);                 // exact error of p*hi
+    const float r = ph - 2.0f * rintf(0.5f * ph);      // exact, |r| <= 1
+    sincospif(r + fmaf(p, lo, pe), &s, &c);
 }
 
 // ----------------------------------------------------------------- mbarrier / bulk copy
@@ -176,6 +181,17 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
         "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// Same without an L2 policy (data that may be read again stays cacheable).
+__device__ __forceinline__ void bulk_load_plain(void *dst, const void *src, uint32_t bytes,
+                                                uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
 }
 

@@ -19,26 +19,32 @@ cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, f
                                void *ws, void *scratch, cudaStream_t st);
 
 // top-k: scratch holds per-slice candidates when NS is large; zero_words
-// (nullable) are cleared by the first CTA (used to reset attention tickets)
+// (nullable) are cleared by the first CTA (used to reset attention tickets);
+// rope_tab (nullable) is filled by spare CTAs of the same launch
 size_t topk_ws_bytes(const Geom &geo);
 cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void *scratch,
-                        uint32_t *zero_words, int nzero, cudaStream_t st);
+                        uint32_t *zero_words, int nzero, float2 *rope_tab, cudaStream_t st);
 
 cudaError_t launch_gather_rope(const Geom &geo, const void *kc, const void *vc, const void *kcur,
                                const void *vcur, const int32_t *sel, float *kw, float *vw,
                                int32_t *win_len, cudaStream_t st);
 
 struct AttnPlan {
+    bool decode;   // warp kernel (<= 8 query rows per KV head) or tile kernel
     int QB, nqb, nsplit;
 };
 AttnPlan attn_plan(const Geom &geo);
 // bytes of tickets (256-aligned, reported separately) + split-K partials
-size_t attend_ws_bytes(const Geom &geo, size_t *ticket_bytes);
-// virt = true: keys/values read from the un-rotated cache through sel;
-// virt = false: from the materialised fp32 window (kw, vw, win_len).
+// (accumulators, then (max, sum) pairs at *ml_off)
+size_t attend_ws_bytes(const Geom &geo, size_t *ticket_bytes, size_t *ml_off);
+// bytes of the per-step RoPE cos/sin table (Wmax x d/2 float2)
+size_t rope_table_bytes(const Geom &geo);
+// virt = true: keys/values read from the un-rotated cache through sel and
+// rotated with rope_tab; virt = false: from the materialised fp32 window.
 cudaError_t launch_attend(const Geom &geo, const void *q, const float *kw, const float *vw,
                           const int32_t *win_len, const void *kc, const void *vc,
-                          const void *kcur, const void *vcur, const int32_t *sel, float *out,
-                          void *scratch, bool virt, cudaStream_t st);
+                          const void *kcur, const void *vcur, const int32_t *sel,
+                          const float2 *rope_tab, float *out, void *scratch, void *ws, bool virt,
+                          cudaStream_t st);
 
 }  // namespace reatt

@@ -37,12 +37,37 @@ int num_sms()
 
 namespace {
 
-constexpr int kConsumerWarps = 8;
+// Ring shape (compile-time; the defaults are the measured best on B200).
+#ifndef REATT_SCAN_CWARPS
+#define REATT_SCAN_CWARPS 16     // consumer warps per CTA
+#endif
+#ifndef REATT_SCAN_RING_KB
+#define REATT_SCAN_RING_KB 192   // shared-memory ring per CTA
+#endif
+#ifndef REATT_SCAN_CPS
+#define REATT_SCAN_CPS 1         // CTAs per SM
+#endif
+#ifndef REATT_SCAN_SUB
+#define REATT_SCAN_SUB 2         // 32-token passes per ring stage
+#endif
+constexpr int kConsumerWarps = REATT_SCAN_CWARPS;
 constexpr int kConsumers = 32 * kConsumerWarps;
 constexpr int kScanThreads = kConsumers + 32;       // + one producer warp
-constexpr int kRingBytes = 192 * 1024;
-constexpr int kMaxItemSpans = 4096;
-constexpr int kPassTok = 32;                          // tokens per ring stage
+constexpr int kRingBytes = REATT_SCAN_RING_KB * 1024;
+constexpr int kCtasPerSm = REATT_SCAN_CPS;
+constexpr int kSub = REATT_SCAN_SUB;
+constexpr int kMaxItemSpans = 4096 / kCtasPerSm;
+constexpr int kPassTok = 32;                          // tokens per consumer pass
+constexpr int kStageTok = kPassTok * kSub;            // tokens per ring stage
+
+constexpr int gcd(int a, int b) { return b == 0 ? a : gcd(b, a % b); }
+// Largest warp count (halving from cw) whose fixed stage map leaves >= 2 stages.
+constexpr int eff_warps(int stages_raw, int cw)
+{
+    return (cw <= 1 || stages_raw / (cw / gcd(cw, kSub)) * (cw / gcd(cw, kSub)) >= 2)
+               ? cw
+               : eff_warps(stages_raw, cw / 2);
+}
 
 template <typename T, int D>
 struct ScanShape {
@@ -50,11 +75,23 @@ struct ScanShape {
     static constexpr int kLpt = kRowBytes / 16;       // lanes per token row
     static constexpr int kNg = 32 / kLpt;             // rows per load round
     static constexpr int kVec = Elem<T>::kVec;        // elements per lane load
-    static constexpr int kStageBytes = kPassTok * kRowBytes;
-    static constexpr int kStages = kRingBytes / kStageBytes;
+    static constexpr int kPassBytes = kPassTok * kRowBytes;
+    static constexpr int kStageBytes = kStageTok * kRowBytes;
+    // Pass slot (stage, j) of ring use u is consumed by warp (st*kSub + j) %
+    // kConsumerWarps with st = stage + u*kStages.  The stage count is a
+    // multiple of kWarpPeriod so that warp is the same for every use: each
+    // full barrier then has a single waiter that takes its phases in order,
+    // and a parity wait can never be two phases ahead (where it would pass at
+    // once on the stale parity).
+    // (Wide rows with many warps: fewer warps consume, the rest idle.)
+    static constexpr int kCW = eff_warps(kRingBytes / kStageBytes, kConsumerWarps);
+    static constexpr int kWarpPeriod = kCW / gcd(kCW, kSub);
+    static constexpr int kStages = kRingBytes / kStageBytes / kWarpPeriod * kWarpPeriod;
     static constexpr size_t kSmem = size_t(kRingBytes) + 2 * kStages * sizeof(uint64_t) +
                                     kMaxItemSpans * sizeof(uint32_t) + D * sizeof(float) + 16;
     static_assert(kLpt * kNg == 32, "row must split evenly over a warp");
+    static_assert(kStages >= 2, "ring too small");
+    static_assert((kStages * kSub) % kCW == 0, "stage -> warp map must be fixed");
 };
 
 // Work of one CTA: global span ids [gs, ge) over the flattened (b*Hkv+h, span)
@@ -80,7 +117,7 @@ __device__ __forceinline__ bool next_item(const Geom &geo, int64_t &gs, int64_t 
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kScanThreads, 1)
+__global__ void __launch_bounds__(kScanThreads, kCtasPerSm)
 scan_decode_kernel(Geom geo, const T *__restrict__ q, const T *__restrict__ kc,
                    float *__restrict__ scores, void *ws, int64_t spans_per_cta)
 {
@@ -103,7 +140,7 @@ scan_decode_kernel(Geom geo, const T *__restrict__ q, const T *__restrict__ kc,
         abort_flag = 0;
         for (int s = 0; s < Sh::kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], kSub);   // one release per pass slot
         }
         mbar_init_fence();
     }
@@ -112,45 +149,60 @@ scan_decode_kernel(Geom geo, const T *__restrict__ q, const T *__restrict__ kc,
     if (warp == kConsumerWarps) {
         // ------------------------------------------------ producer (one thread)
         if (lane == 0) {
+            // Stage index and use parity advance incrementally (no divisions in
+            // the issue loop: one thread issues every copy of the CTA).
             const uint64_t pol = l2_evict_first_policy();
-            int64_t n = 0, gs = cta_begin;
+            int stage = 0;
+            uint32_t phase = 0;         // parity of the current use of `stage`
+            bool wrapped = false;       // every stage has been used once
+            int64_t gs = cta_begin;
             Item it;
             bool stop = false;
             while (!stop && next_item(geo, gs, cta_end, it)) {
-                const T *base = kc + it.bh * geo.T * D;
-                for (int64_t t = it.t_begin; t < it.t_end; t += kPassTok, ++n) {
-                    const int stage = int(n % Sh::kStages);
-                    if (n >= Sh::kStages) {
-                        const uint32_t par = uint32_t((n / Sh::kStages - 1) & 1);
+                const T *src = kc + (it.bh * geo.T + it.t_begin) * D;
+                for (int64_t t = it.t_begin; t < it.t_end; t += kStageTok, src += kStageTok * D) {
+                    if (wrapped) {
                         if (*(volatile int *)&abort_flag ||
-                            !mbar_wait_bounded(&empty[stage], par, kWaitLimitNs)) {
+                            !mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs)) {
                             report_status(ws, REATT_ETIMEOUT);
                             *(volatile int *)&abort_flag = 1;
                             stop = true;
                             break;
                         }
                     }
-                    int64_t ntok = it.t_end - t;
-                    if (ntok > kPassTok) ntok = kPassTok;
-                    const uint32_t bytes = uint32_t(ntok) * Sh::kRowBytes;
+                    const int64_t left = it.t_end - t;
+                    const uint32_t bytes =
+                        uint32_t(left < kStageTok ? left : kStageTok) * Sh::kRowBytes;
                     mbar_arrive_expect_tx(&full[stage], bytes);
-                    bulk_load(ring + size_t(stage) * Sh::kStageBytes, base + t * D, bytes,
-                              &full[stage], pol);
+                    bulk_load(ring + stage * Sh::kStageBytes, src, bytes, &full[stage], pol);
+                    if (++stage == Sh::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                        wrapped = true;
+                    }
                 }
             }
-            // Drain: every issued copy has landed before the CTA may exit.
-            const int64_t first = n > Sh::kStages ? n - Sh::kStages : 0;
-            for (int64_t m = first; m < n; ++m)
-                if (!mbar_wait_bounded(&full[m % Sh::kStages], uint32_t((m / Sh::kStages) & 1),
-                                       kWaitLimitNs))
+            // Drain: every issued copy has landed before the CTA may exit.  The
+            // last use of each stage (the most recent kStages issues) is waited
+            // on with that use's parity.
+            for (int k2 = 0; k2 < Sh::kStages; ++k2) {
+                if (--stage < 0) {
+                    stage = Sh::kStages - 1;
+                    if (!wrapped) break;      // fewer than kStages issues in all
+                    phase ^= 1u;
+                }
+                if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs))
                     report_status(ws, REATT_ETIMEOUT);
+            }
         }
         return;
     }
 
-    // ---------------------------------------------------- consumers (8 warps)
+    // ---------------------------------------------------- consumers
     const int gq = lane / Sh::kLpt, p = lane % Sh::kLpt;
-    int64_t n = 0, gs = cta_begin;
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t gs = cta_begin;
     Item it;
     while (next_item(geo, gs, cta_end, it)) {
         // fp32 sum of the group's query vectors (query position 0)
@@ -171,67 +223,81 @@ scan_decode_kernel(Geom geo, const T *__restrict__ q, const T *__restrict__ kc,
         for (int e = 0; e < Sh::kVec; ++e)
             qv[e] = qs[p * Sh::kVec + e];
 
-        for (int64_t t = it.t_begin; t < it.t_end; t += kPassTok, ++n) {
-            if (int(n % kConsumerWarps) != warp)
-                continue;
-            // warp-uniform abort / wait outcome (the shuffles below need all lanes)
-            if (__any_sync(0xffffffffu, *(volatile int *)&abort_flag != 0))
-                continue;
-            const int stage = int(n % Sh::kStages);
-            const bool ok =
-                mbar_wait_bounded(&full[stage], uint32_t((n / Sh::kStages) & 1), kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) {
-                    report_status(ws, REATT_ETIMEOUT);
-                    *(volatile int *)&abort_flag = 1;
+        for (int64_t t = it.t_begin; t < it.t_end; t += kStageTok) {
+            const uint32_t par = phase;
+            const int st_now = stage;
+            if (++stage == Sh::kStages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+            // fixed map: slot j of ring stage s belongs to warp (s*kSub + j) % kCW
+#pragma unroll
+            for (int j = 0; j < kSub; ++j) {
+                if ((st_now * kSub + j) % Sh::kCW != warp)
+                    continue;
+                // warp-uniform abort / wait outcome (the shuffles below need all lanes)
+                if (__any_sync(0xffffffffu, *(volatile int *)&abort_flag != 0))
+                    continue;
+                const bool ok = mbar_wait_bounded(&full[st_now], par, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0) {
+                        report_status(ws, REATT_ETIMEOUT);
+                        *(volatile int *)&abort_flag = 1;
+                    }
+                    continue;
                 }
-                continue;
-            }
-            const uint8_t *sb = ring + size_t(stage) * Sh::kStageBytes;
-            float acc[Sh::kLpt];
-#pragma unroll
-            for (int r = 0; r < Sh::kLpt; ++r) {
-                const uint4 raw = *reinterpret_cast<const uint4 *>(
-                    sb + (r * Sh::kNg + gq) * Sh::kRowBytes + p * 16);
-                float e[Sh::kVec];
-                Elem<T>::unpack(raw, e);
-                float a = 0.f;
-#pragma unroll
-                for (int i = 0; i < Sh::kVec; ++i)
-                    a = fmaf(qv[i], e[i], a);
-                acc[r] = a;
-            }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&empty[stage]);   // the stage is in registers: hand it back
-
-            // Transposed reduction over the kLpt lanes of a row group: after
-            // it lane (gq, p) holds the full dot product of row p*kNg + gq.
-#pragma unroll
-            for (int o = Sh::kLpt / 2; o >= 1; o >>= 1) {
-                const bool upper = (p & o) != 0;
-#pragma unroll
-                for (int i = 0; i < o; ++i) {
-                    const float send = upper ? acc[i] : acc[i + o];
-                    const float keep = upper ? acc[i + o] : acc[i];
-                    acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                const int64_t tp = t + int64_t(j) * kPassTok;
+                int ntok = int(it.t_end - tp);
+                if (ntok > kPassTok) ntok = kPassTok;
+                if (ntok <= 0) {   // empty slot of a short last stage: release only
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[st_now]);
+                    continue;
                 }
-            }
-            int ntok = int(it.t_end - t);
-            if (ntok > kPassTok) ntok = kPassTok;
-            const int row = p * Sh::kNg + gq;
-            const bool valid = row < ntok;
-            const int moff = int(t - geo.G);                 // middle offset of row 0
-            const int sfirst = moff / geo.S, slast = (moff + ntok - 1) / geo.S;
-            if (sfirst == slast) {
-                float m = valid ? acc[0] : -INFINITY;
+                const uint8_t *sb = ring + st_now * Sh::kStageBytes + j * Sh::kPassBytes;
+                float acc[Sh::kLpt];
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1)
-                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                for (int r = 0; r < Sh::kLpt; ++r) {
+                    const uint4 raw = *reinterpret_cast<const uint4 *>(
+                        sb + (r * Sh::kNg + gq) * Sh::kRowBytes + p * 16);
+                    float e[Sh::kVec];
+                    Elem<T>::unpack(raw, e);
+                    float a = 0.f;
+#pragma unroll
+                    for (int i = 0; i < Sh::kVec; ++i)
+                        a = fmaf(qv[i], e[i], a);
+                    acc[r] = a;
+                }
+                __syncwarp();
                 if (lane == 0)
-                    atomicMax(&smax[sfirst - int(it.s0)], order_code(m));
-            } else if (valid) {
-                atomicMax(&smax[(moff + row) / geo.S - int(it.s0)], order_code(acc[0]));
+                    mbar_arrive(&empty[st_now]);   // the pass is in registers: hand it back
+
+                // Transposed reduction over the kLpt lanes of a row group: after
+                // it lane (gq, p) holds the full dot product of row p*kNg + gq.
+#pragma unroll
+                for (int o = Sh::kLpt / 2; o >= 1; o >>= 1) {
+                    const bool upper = (p & o) != 0;
+#pragma unroll
+                    for (int i = 0; i < o; ++i) {
+                        const float send = upper ? acc[i] : acc[i + o];
+                        const float keep = upper ? acc[i + o] : acc[i];
+                        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                    }
+                }
+                const int row = p * Sh::kNg + gq;
+                const bool valid = row < ntok;
+                const int moff = int(tp - geo.G);                // middle offset of row 0
+                const int sfirst = moff / geo.S, slast = (moff + ntok - 1) / geo.S;
+                if (sfirst == slast) {
+                    float m = valid ? acc[0] : -INFINITY;
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1)
+                        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                    if (lane == 0)
+                        atomicMax(&smax[sfirst - int(it.s0)], order_code(m));
+                } else if (valid) {
+                    atomicMax(&smax[(moff + row) / geo.S - int(it.s0)], order_code(acc[0]));
+                }
             }
         }
         named_sync(1, kConsumers);
@@ -332,7 +398,7 @@ cudaError_t launch_decode(const Geom &geo, const void *q, const void *kc, float 
 {
     using Sh = ScanShape<T, D>;
     const int64_t total = int64_t(geo.B) * geo.Hkv * geo.NS;
-    int grid = num_sms();
+    int grid = num_sms() * kCtasPerSm;
     if (total < grid) grid = int(total);
     const int64_t per = (total + grid - 1) / grid;
     grid = int((total + per - 1) / per);
