@@ -48,6 +48,12 @@ CASES = {
                                      n_needles=0, seed=20),
     "prefill_bf16_c70": LLAMA.replace(name="c70", Hq=4, Hkv=1, C=70, T=3000, G=8, L=64, S=32,
                                       k=5, n_needles=0, seed=23),
+    "prefill_bf16_g2_d64_c300": LLAMA.replace(name="c300", Hq=4, Hkv=2, d=64, C=300, T=5000,
+                                              G=8, L=100, S=16, k=20, n_needles=0, seed=24),
+    "prefill_bf16_g1_c130_s8": LLAMA.replace(name="c130", Hq=2, Hkv=2, C=130, T=2600, G=8,
+                                             L=64, S=8, k=30, n_needles=0, seed=25),
+    "prefill_bf16_s64_fallback": LLAMA.replace(name="s64", Hq=4, Hkv=1, C=9, T=3000, G=8, L=64,
+                                               S=64, k=5, n_needles=0, seed=26),
     "two_level_topk": LLAMA.replace(name="big_ns", Hq=2, Hkv=1, d=64, T=200000, G=32, L=256,
                                     S=8, k=100, n_needles=4, seed=21),
     "batch3_large_s": TINY.replace(name="b3", B=3, Hq=2, Hkv=1, T=5000, G=2, L=40, S=100, k=3,

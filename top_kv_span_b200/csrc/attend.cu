@@ -373,6 +373,7 @@ attend_decode_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid < D / 2) freq[tid] = make_float2(geo.rope_hi[tid], geo.rope_lo[tid]);
+    pdl_wait();
     __syncthreads();
     const int split = blockIdx.x;
     const int64_t bh = blockIdx.z;
@@ -588,26 +589,30 @@ struct TmaShape {
 static_assert(kTmaStages % kTmaCW == 0, "stage -> warp map must be fixed");
 
 // Chunk of window rows starting at p: its length (contiguous source run).
-__device__ __forceinline__ int chunk_len(const Geom &geo, const WinMap &m, int64_t p, int64_t kend,
+__device__ __forceinline__ int chunk_len(const Geom &geo, const WinMap &m, int p, int kend,
                                          int chunk)
 {
-    const int64_t g_end = m.g_end, nsel = m.nsel_rows, nloc = m.n_loc;
-    int64_t end;
+    const int g_end = int(m.g_end), nsel = int(m.nsel_rows), nloc = int(m.n_loc);
+    int end;
     if (p < g_end) {
         end = g_end;
     } else if (p < g_end + nsel) {
-        const int64_t j = (p - g_end) / geo.S;
+        const int j = (p - g_end) / geo.S;
         end = g_end + (j + 1) * geo.S;
         if (end > g_end + nsel) end = g_end + nsel;
     } else if (p < g_end + nsel + nloc) {
         end = g_end + nsel + nloc;
     } else {
-        end = m.W;
+        end = int(m.W);
     }
     if (end > kend) end = kend;
     if (end > p + chunk) end = p + chunk;
-    return int(end - p);
+    return end - p;
 }
+
+// The chosen span ids a CTA's key range touches, staged in shared memory so
+// the producer's address computations do not wait on global loads.
+constexpr int kSelCache = 512;
 
 template <typename T, int D, int RP>
 __global__ void __launch_bounds__((kTmaCW + 1) * 32, 1)
@@ -618,6 +623,9 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
     constexpr int PD = D / 64;            // RoPE pairs per lane
     constexpr int KB = 32 / RP;           // keys per reduction batch
     constexpr int RB = Sh::kRowBytes;
+    constexpr int CH = Sh::kChunk;
+    constexpr int EB = Elem<T>::kBytes;
+    static_assert(kTmaStages == kTmaCW, "warp w owns ring stage w");
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Sh::kRing);
@@ -627,19 +635,11 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
     float *s_l = s_m + kTmaCW * RP;
     __shared__ float f_m[RP], f_l[RP];
     __shared__ float2 freq[D / 2];
+    __shared__ __align__(16) float q_s[RP][D];     // rotated, scaled queries
     __shared__ int is_last, abort_flag;
+    __shared__ int32_t sel_s[kSelCache];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int split = blockIdx.x;
-    const int64_t bh = blockIdx.z;
-    const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv);
-    const int nrows = geo.g * geo.C;
-    const int32_t *sel_bh = a.sel + bh * geo.k;
-    const WinMap m = make_winmap(geo, sel_bh);
-    const int64_t W = m.W, qpos0 = W - geo.C;
-    int64_t kbeg, kend;
-    split_range(geo, W, a.nsplit, split, 0, nrows, Sh::kChunk, kbeg, kend);
-
     if (tid == 0) {
         abort_flag = 0;
         for (int s = 0; s < kTmaStages; ++s) {
@@ -649,46 +649,94 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
         mbar_init_fence();
     }
     if (tid < D / 2) freq[tid] = make_float2(geo.rope_hi[tid], geo.rope_lo[tid]);
+    pdl_wait();   // the selection (and tickets) come from the preceding kernels
+
+    const int split = blockIdx.x;
+    const int64_t bh = blockIdx.z;
+    const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv);
+    const int nrows = geo.g * geo.C;
+    const int32_t *sel_bh = a.sel + bh * geo.k;
+    const WinMap m = make_winmap(geo, sel_bh);
+    const int64_t W = m.W, qpos0 = W - geo.C;
+    int64_t kbeg64, kend64;
+    split_range(geo, W, a.nsplit, split, 0, nrows, CH, kbeg64, kend64);
+    const int kbeg = int(kbeg64), kend = int(kend64);
+    // span ids of the chosen part inside [kbeg, kend)
+    const int g_end = int(m.g_end), nsel = int(m.nsel_rows), nloc = int(m.n_loc);
+    int j0 = 0, jn = 0;
+    {
+        const int lo = kbeg > g_end ? kbeg : g_end;
+        const int hi = kend < g_end + nsel ? kend : g_end + nsel;
+        if (lo < hi) {
+            j0 = (lo - g_end) / geo.S;
+            jn = (hi - 1 - g_end) / geo.S - j0 + 1;
+        }
+    }
+    const bool sel_cached = jn <= kSelCache;
+    if (sel_cached)
+        for (int j = tid; j < jn; j += blockDim.x) sel_s[j] = sel_bh[j0 + j];
+    __syncthreads();   // freq visible to the query rotation
+    for (int x = tid; x < RP * (D / 2); x += blockDim.x) {
+        const int rr = x / (D / 2), i = x % (D / 2);
+        float lo = 0.f, hi = 0.f;
+        if (rr < nrows) query_pair<T, D>(geo, freq, a.q, b, h, rr, qpos0, i, lo, hi);
+        q_s[rr][i] = lo;
+        q_s[rr][i + D / 2] = hi;
+    }
     __syncthreads();
 
+    const int nchunks = kend > kbeg ? (kend - kbeg + CH - 1) / CH : 0;
     if (warp == kTmaCW) {
         // ------------------------------------------------ producer (one thread)
+        // chunk ci = window rows [kbeg + ci*CH, +CH) -> stage ci % kTmaStages;
+        // a chunk crossing a region boundary is copied as several runs
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            bool wrapped = false;
-            for (int64_t p = kbeg; p < kend;) {
-                const int n = chunk_len(geo, m, p, kend, Sh::kChunk);
-                if (wrapped && (*(volatile int *)&abort_flag ||
-                                !mbar_wait_bounded(&empty[stage], phase ^ 1u, kWaitLimitNs))) {
+            int issued = 0;
+            for (int ci = 0; ci < nchunks; ++ci, ++issued) {
+                const int stage = ci % kTmaStages;
+                if (ci >= kTmaStages &&
+                    (*(volatile int *)&abort_flag ||
+                     !mbar_wait_bounded(&empty[stage], uint32_t(((ci / kTmaStages) - 1) & 1),
+                                        kWaitLimitNs))) {
                     report_status(ws, REATT_ETIMEOUT);
                     *(volatile int *)&abort_flag = 1;
                     break;
                 }
-                const int64_t off = win_row_offset(geo, m, sel_bh, bh, int(p), D);
-                const bool cur = (off >> 62) != 0;
-                const int64_t o = off & ~(int64_t(1) << 62);
-                const uint32_t bytes = uint32_t(n) * RB;
+                const int p0 = kbeg + ci * CH;
+                const int n = kend - p0 < CH ? kend - p0 : CH;
                 uint8_t *dst = ring + stage * Sh::kStageBytes;
-                mbar_arrive_expect_tx(&full[stage], 2 * bytes);
-                bulk_load_plain(dst, (cur ? kcur : kc) + o, bytes, &full[stage]);
-                bulk_load_plain(dst + Sh::kChunk * RB, (cur ? vcur : vc) + o, bytes, &full[stage]);
-                p += n;
-                if (++stage == kTmaStages) {
-                    stage = 0;
-                    phase ^= 1u;
-                    wrapped = true;
+                mbar_arrive_expect_tx(&full[stage], 2u * uint32_t(n) * RB);
+                for (int p = p0; p < p0 + n;) {
+                    const int r = chunk_len(geo, m, p, p0 + n, CH);
+                    bool cur = false;
+                    int64_t o;
+                    if (p < g_end) {
+                        o = (bh * geo.T + p) * D;
+                    } else if (p - g_end < nsel) {
+                        const int q = p - g_end, j = q / geo.S, off = q - j * geo.S;
+                        int sp = sel_cached ? sel_s[j - j0] : sel_bh[j];
+                        sp = sp < 0 ? 0 : (sp >= int(geo.NS) ? int(geo.NS) - 1 : sp);
+                        int srow = geo.G + sp * geo.S + off;
+                        if (srow >= int(geo.T)) srow = int(geo.T) - 1;
+                        o = (bh * geo.T + srow) * D;
+                    } else if (p - g_end - nsel < nloc) {
+                        o = (bh * geo.T + m.loc_begin + (p - g_end - nsel)) * D;
+                    } else {
+                        cur = true;
+                        o = (bh * geo.C + (p - g_end - nsel - nloc)) * D;
+                    }
+                    const uint32_t bytes = uint32_t(r) * RB;
+                    bulk_load_plain(dst + (p - p0) * RB, (cur ? kcur : kc) + o, bytes, &full[stage]);
+                    bulk_load_plain(dst + (CH + p - p0) * RB, (cur ? vcur : vc) + o, bytes,
+                                    &full[stage]);
+                    p += r;
                 }
             }
-            for (int k2 = 0; k2 < kTmaStages; ++k2) {   // drain the copies in flight
-                if (--stage < 0) {
-                    stage = kTmaStages - 1;
-                    if (!wrapped) break;
-                    phase ^= 1u;
-                }
-                if (!mbar_wait_bounded(&full[stage], phase, kWaitLimitNs))
+            // drain: the last use of every stage that was issued
+            for (int ci = issued - 1; ci >= 0 && ci >= issued - kTmaStages; --ci)
+                if (!mbar_wait_bounded(&full[ci % kTmaStages], uint32_t((ci / kTmaStages) & 1),
+                                       kWaitLimitNs))
                     report_status(ws, REATT_ETIMEOUT);
-            }
         }
     } else {
         // ---------------------------------------------------- consumers
@@ -700,8 +748,8 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
             rope_cs(1, freq[i].x, freq[i].y, step[e].x, step[e].y);
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
-                qlo[r][e] = qhi[r][e] = 0.f;
-                if (r < nrows) query_pair<T, D>(geo, freq, a.q, b, h, r, qpos0, i, qlo[r][e], qhi[r][e]);
+                qlo[r][e] = q_s[r][i];
+                qhi[r][e] = q_s[r][i + D / 2];
             }
         }
         const int my_r = lane % RP;
@@ -716,39 +764,29 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
         }
         float m_own = -INFINITY;
 
-        int stage = 0, ci = 0;
-        uint32_t phase = 0;
-        for (int64_t p = kbeg; p < kend; ++ci) {
-            const int n = chunk_len(geo, m, p, kend, Sh::kChunk);
-            const int64_t pc = p;
-            const int st_now = stage;
-            const uint32_t par = phase;
-            p += n;
-            if (++stage == kTmaStages) {
-                stage = 0;
-                phase ^= 1u;
-            }
-            if ((st_now % kTmaCW) != warp) continue;
-            if (__any_sync(0xffffffffu, *(volatile int *)&abort_flag != 0)) continue;
-            const bool ok = mbar_wait_bounded(&full[st_now], par, kWaitLimitNs);
+        for (int ci = warp; ci < nchunks; ci += kTmaCW) {
+            const int stage = ci % kTmaStages;
+            const int p0 = kbeg + ci * CH;
+            const int n = kend - p0 < CH ? kend - p0 : CH;
+            if (__any_sync(0xffffffffu, *(volatile int *)&abort_flag != 0)) break;
+            const bool ok =
+                mbar_wait_bounded(&full[stage], uint32_t((ci / kTmaStages) & 1), kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) {
                     report_status(ws, REATT_ETIMEOUT);
                     *(volatile int *)&abort_flag = 1;
                 }
-                continue;
+                break;
             }
-            const uint8_t *kb = ring + st_now * Sh::kStageBytes;
-            const uint8_t *vb = kb + Sh::kChunk * RB;
-            for (int sb = 0; sb < n; sb += KB) {
-                // anchor cos/sin at the first key of the sub-batch
-                float2 cs[PD];
+            const uint8_t *kb = ring + stage * Sh::kStageBytes;
+            const uint8_t *vb = kb + CH * RB;
+            float2 cs[PD];   // RoPE of this lane's pairs at the chunk's first row
 #pragma unroll
-                for (int e = 0; e < PD; ++e) {
-                    const int i = PD * lane + e;
-                    rope_cs(pc + sb, freq[i].x, freq[i].y, cs[e].x, cs[e].y);
-                }
-                constexpr int EB = Elem<T>::kBytes;
+            for (int e = 0; e < PD; ++e) {
+                const int i = PD * lane + e;
+                rope_cs(p0, freq[i].x, freq[i].y, cs[e].x, cs[e].y);
+            }
+            for (int sb = 0; sb < n; sb += KB) {
                 float part[32];
 #pragma unroll
                 for (int kk = 0; kk < KB; ++kk) {
@@ -793,7 +831,7 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
                     }
                 }
                 const int my_row = sb + lane / RP;
-                const int64_t my_p = pc + my_row;
+                const int64_t my_p = int64_t(p0) + my_row;
                 const float x = (my_row < n && my_p <= my_lim) ? part[0] : -INFINITY;
                 float bm = x;
 #pragma unroll
@@ -842,7 +880,7 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st_now]);   // chunk consumed: hand the stage back
+            if (lane == 0) mbar_arrive(&empty[stage]);   // chunk consumed: hand the stage back
         }
         // this warp's state to shared memory
 #pragma unroll
@@ -901,7 +939,8 @@ cudaError_t launch_staged_attn(const Geom &geo, const AttnArgs &a, int RP, const
         cudaError_t e =                                                                        \
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)); \
         if (e != cudaSuccess) return e;                                                        \
-        kern<<<grid, (kTmaCW + 1) * 32, smem, st>>>(geo, a, k, v, kq, vq, ws);                 \
+        e = launch_pdl(kern, grid, dim3((kTmaCW + 1) * 32), smem, st, geo, a, k, v, kq, vq, ws); \
+        if (e != cudaSuccess) return e;                                                        \
     } while (0)
     switch (RP) {
     case 1: REATT_STAGED(1); break;
@@ -1023,7 +1062,7 @@ attend_tile_kernel(Geom geo, AttnArgs a, KvSource<T, D, VIRT> src)
     constexpr int KS = Sm::kKS;
     static_assert(NITEM >= 1 && kKT * HV % kAttnThreads == 0, "tile shape");
     static_assert(kAttnThreads % kKT == 0 && QB % 4 == 0, "tile shape");
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     float *Qs = reinterpret_cast<float *>(smem);
     float *Ks = reinterpret_cast<float *>(smem + Sm::kQ);
     float *Vs = reinterpret_cast<float *>(smem + Sm::kQ + Sm::kK);
@@ -1036,6 +1075,7 @@ attend_tile_kernel(Geom geo, AttnArgs a, KvSource<T, D, VIRT> src)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid < D / 2) freq[tid] = make_float2(geo.rope_hi[tid], geo.rope_lo[tid]);
+    pdl_wait();
     __syncthreads();
     const int split = blockIdx.x, qb = blockIdx.y;
     const int64_t bh = blockIdx.z;
@@ -1202,7 +1242,8 @@ cudaError_t launch_tile(const Geom &geo, const AttnArgs &a, const KvSource<T, D,
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Sm::kTotal));
     if (e != cudaSuccess) return e;
     dim3 grid(unsigned(a.nsplit), unsigned(a.nqb), unsigned(geo.B * geo.Hkv));
-    kern<<<grid, kAttnThreads, Sm::kTotal, st>>>(geo, a, src);
+    e = launch_pdl(kern, grid, dim3(kAttnThreads), Sm::kTotal, st, geo, a, src);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -1215,8 +1256,11 @@ cudaError_t launch_decode_attn(const Geom &geo, const AttnArgs &a, int RP, const
     const T *k = static_cast<const T *>(kc), *v = static_cast<const T *>(vc);
     const T *kq = static_cast<const T *>(kcur), *vq = static_cast<const T *>(vcur);
 #define REATT_DEC(RPV)                                                                         \
-    attend_decode_kernel<T, D, RPV, VIRT><<<grid, kDecWarps * 32, 0, st>>>(geo, a, k, v, kq,   \
-                                                                            vq, kw, vw)
+    do {                                                                                       \
+        cudaError_t e = launch_pdl(attend_decode_kernel<T, D, RPV, VIRT>, grid,                \
+                                   dim3(kDecWarps * 32), 0, st, geo, a, k, v, kq, vq, kw, vw); \
+        if (e != cudaSuccess) return e;                                                        \
+    } while (0)
     switch (RP) {
     case 1: REATT_DEC(1); break;
     case 2: REATT_DEC(2); break;

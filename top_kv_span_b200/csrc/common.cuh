@@ -195,6 +195,13 @@ __device__ __forceinline__ void bulk_load_plain(void *dst, const void *src, uint
         : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor ends; pdl_wait() blocks
+// until the predecessor grid has completed and its writes are visible (a
+// no-op for an ordinary launch); pdl_trigger() lets the successor launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_sync(int id, int count)
 {

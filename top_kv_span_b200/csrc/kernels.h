@@ -5,9 +5,31 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace reatt {
+
+// Launch with programmatic stream serialization: the kernel may begin while
+// its predecessor in the stream finishes; it must call pdl_wait() before
+// touching anything the predecessor writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 inline bool geo_is_bf16(const Geom &g) { return g.dtype == REATT_BF16; }
 
@@ -17,6 +39,12 @@ int num_sms();
 size_t score_spans_ws_bytes(const Geom &geo);
 cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, float *scores,
                                void *ws, void *scratch, cudaStream_t st);
+
+// prefill span scoring on tcgen05 (bf16, C > 1, S divides 32)
+bool prefill_tc_eligible(const Geom &geo);
+size_t prefill_tc_ws_bytes(const Geom &geo);
+cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, float *scores,
+                              void *ws, void *scratch, cudaStream_t st);
 
 // top-k: scratch holds per-slice candidates when NS is large; zero_words
 // (nullable) are cleared by the first CTA (used to reset attention tickets);

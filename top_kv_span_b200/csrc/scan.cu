@@ -136,6 +136,7 @@ scan_decode_kernel(Geom geo, const T *__restrict__ q, const T *__restrict__ kc,
     int64_t cta_end = cta_begin + spans_per_cta;
     if (cta_end > total) cta_end = total;
 
+    pdl_trigger();   // the top-k may launch now; it waits for this grid to finish
     if (tid == 0) {
         abort_flag = 0;
         for (int s = 0; s < Sh::kStages; ++s) {
@@ -431,7 +432,9 @@ cudaError_t launch_multi(const Geom &geo, const void *q, const void *kc, float *
 size_t score_spans_ws_bytes(const Geom &geo)
 {
     if (geo.C <= 1) return 0;
-    return size_t(geo.B) * geo.Hkv * geo.C * geo.d * sizeof(float);
+    const size_t qsum = size_t(geo.B) * geo.Hkv * geo.C * geo.d * sizeof(float);
+    const size_t terms = prefill_tc_ws_bytes(geo);
+    return qsum > terms ? qsum : terms;
 }
 
 cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, float *scores,
@@ -445,6 +448,8 @@ cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, f
         return geo_is_bf16(geo) ? launch_decode<uint16_t, 64>(geo, q, kc, scores, ws, st)
                                 : launch_decode<float, 64>(geo, q, kc, scores, ws, st);
     }
+    if (prefill_tc_eligible(geo))   // tensor-core contraction (tcgen05 / TMEM)
+        return launch_prefill_tc(geo, q, kc, scores, ws, scratch, st);
     float *qsum = static_cast<float *>(scratch);
     if (geo.d == 128)
         return geo_is_bf16(geo) ? launch_multi<uint16_t, 128>(geo, q, kc, scores, qsum, st)

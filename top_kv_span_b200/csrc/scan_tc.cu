@@ -1,0 +1,447 @@
+// Prefill span scoring on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// For a chunk of C > 1 queries (chunked prefill) the span score of the
+// decoding pseudocode becomes a contraction (ReAttention OpenReview
+// discussion, "Prefilling Phase": score = query . key[global:-local]^T over
+// the whole chunk):
+//   s[t] = max_c sum_{j in group(h)} q[b,j,c,:] . k[b,h,t,:],
+//   span_score = max over the span's tokens.
+// The group's query vectors are summed in fp32 (linearity), and the fp32 sum
+// is split into bf16 hi + lo terms (hi = bf16(s), lo = bf16(s - hi)); both
+// terms accumulate into the same fp32 TMEM tile, so the product is exact to
+// ~2^-17 relative -- one bf16 rounding of the sum would not be.  With g <= 2
+// query heads per KV head the raw bf16 heads are the terms instead (exact).
+//
+// Kernel: one CTA per SM, persistent over (head, 128-token tile) items.
+//   warp 0  : TMA producer (cp.async.bulk.tensor, 128B swizzle, no multicast)
+//   warp 1  : TMEM allocation; one thread issues tcgen05.mma (M=128 tokens,
+//             N=128 queries, K=16) into two TMEM accumulators in turn
+//   warps 2-5: epilogue -- tcgen05.ld of the accumulator rows (one token row
+//             per thread), max over valid queries, then a segmented warp max
+//             over the span's tokens; only span scores reach global memory.
+// Every wait is bounded; a timeout records REATT_ETIMEOUT in the workspace.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace reatt {
+
+namespace {
+
+constexpr int kTcThreads = 6 * 32;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kTileM = 128;          // tokens per tile = TMEM lanes
+constexpr int kTileN = 128;          // queries per MMA tile = TMEM columns
+constexpr int kQStages = 4;          // query-tile ring
+constexpr uint32_t kTmemCols = 256;  // two accumulators
+constexpr int kBoxBytes = 128 * 128; // one 128-row x 64-element bf16 box (128 B rows)
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] x B[smem desc]^T, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// The mbarrier gets one arrival when every tcgen05 op issued so far by this
+// thread has completed.
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_addr(bar))
+        : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 2-D tiled TMA load (no multicast); x is the innermost (element) coordinate.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+// Shared-memory matrix descriptor: K-major operand in 128-byte-swizzled 8-row
+// atoms (rows of 128 B, 8-row groups 1024 B apart), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(const void *p)
+{
+    const uint64_t addr = smem_addr(p);
+    uint64_t d = (addr >> 4) & 0x3FFFull;    // start address
+    d |= 1ull << 16;                          // leading byte offset (unused: swizzled K-major)
+    d |= uint64_t(1024 >> 4) << 32;           // stride byte offset between 8-row groups
+    d |= 1ull << 46;                          // version
+    d |= 2ull << 61;                          // 128-byte swizzle
+    return d;
+}
+// Instruction descriptor, kind::f16: fp32 D, bf16 A and B, both K-major, M x N.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kTileN >> 3) << 17) |
+                            (uint32_t(kTileM >> 4) << 24);
+
+struct TcArgs {
+    int64_t items;   // BH * ntiles
+    int ntiles;      // 128-token tiles per head
+    int nqt;         // 128-query tiles
+    int nterms;      // bf16 terms per query
+    int cpad;        // nqt * 128
+};
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+                       const __grid_constant__ CUtensorMap qmap, Geom geo, TcArgs ta,
+                       float *__restrict__ scores, void *ws)
+{
+    constexpr int KS = D / 16;             // MMA k-steps over the head width
+    constexpr int NBOX = D / 64;           // 64-element swizzle boxes per row
+    constexpr uint32_t kKBytes = NBOX * kBoxBytes;
+    constexpr uint32_t kQBytes = NBOX * kBoxBytes;
+    extern __shared__ uint8_t smem_raw[];
+    // 128B-swizzled operand tiles want 1024-byte alignment
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint8_t *ksm = smem;
+    uint8_t *qsm = smem + kKBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(qsm + kQStages * kQBytes);
+    uint64_t *kfull = bars, *kempty = bars + 1;
+    uint64_t *qfull = bars + 2, *qempty = qfull + kQStages;
+    uint64_t *accfull = qempty + kQStages, *accempty = accfull + 2, *done = accempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+    __shared__ int abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        abort_flag = 0;
+        mbar_init(kfull, 1);
+        mbar_init(kempty, 1);
+        for (int s = 0; s < kQStages; ++s) {
+            mbar_init(&qfull[s], 1);
+            mbar_init(&qempty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&accfull[s], 1);
+            mbar_init(&accempty[s], 4);   // one arrival per epilogue warp
+        }
+        mbar_init(done, 1);
+        mbar_init_fence();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    auto fail = [&]() {
+        report_status(ws, REATT_ETIMEOUT);
+        *(volatile int *)&abort_flag = 1;
+    };
+    auto aborted = [&]() { return *(volatile int *)&abort_flag != 0; };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t kuse = 0, qn = 0;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; ok && it < ta.items; it += gridDim.x) {
+                const int64_t bh = it / ta.ntiles;
+                const int tile = int(it % ta.ntiles);
+                const int y = int(bh * geo.T + geo.G + int64_t(tile) * kTileM);
+                if (kuse > 0 && (aborted() || !mbar_wait_bounded(kempty, (kuse - 1) & 1, kWaitLimitNs))) {
+                    fail();
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(kfull, kKBytes);
+                for (int bx = 0; bx < NBOX; ++bx) tma_load_2d(ksm + bx * kBoxBytes, &kmap, 64 * bx, y, kfull);
+                ++kuse;
+                for (int qt = 0; ok && qt < ta.nqt; ++qt)
+                    for (int term = 0; term < ta.nterms; ++term, ++qn) {
+                        const int st = int(qn % kQStages);
+                        const uint32_t use = qn / kQStages;
+                        if (use > 0 && (aborted() || !mbar_wait_bounded(&qempty[st], (use - 1) & 1, kWaitLimitNs))) {
+                            fail();
+                            ok = false;
+                            break;
+                        }
+                        const int qy = int((bh * ta.nterms + term) * ta.cpad + int64_t(qt) * kTileN);
+                        mbar_arrive_expect_tx(&qfull[st], kQBytes);
+                        for (int bx = 0; bx < NBOX; ++bx)
+                            tma_load_2d(qsm + st * kQBytes + bx * kBoxBytes, &qmap, 64 * bx, qy,
+                                        &qfull[st]);
+                    }
+            }
+            // drain: the last K load and the last query loads have landed
+            if (kuse > 0 && !mbar_wait_bounded(kfull, (kuse - 1) & 1, kWaitLimitNs)) fail();
+            for (uint32_t m = qn > kQStages ? qn - kQStages : 0; m < qn; ++m)
+                if (!mbar_wait_bounded(&qfull[m % kQStages], (m / kQStages) & 1, kWaitLimitNs)) fail();
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t kuse = 0, qn = 0, an = 0;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; ok && it < ta.items; it += gridDim.x) {
+                if (aborted() || !mbar_wait_bounded(kfull, kuse & 1, kWaitLimitNs)) {
+                    fail();
+                    break;
+                }
+                ++kuse;
+                tc_fence_after();
+                for (int qt = 0; ok && qt < ta.nqt; ++qt, ++an) {
+                    const int acc = int(an & 1);
+                    const uint32_t ause = an >> 1;
+                    if (ause > 0 && (aborted() || !mbar_wait_bounded(&accempty[acc], (ause - 1) & 1, kWaitLimitNs))) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + uint32_t(acc * kTileN);
+                    for (int term = 0; term < ta.nterms; ++term, ++qn) {
+                        const int st = int(qn % kQStages);
+                        if (aborted() || !mbar_wait_bounded(&qfull[st], (qn / kQStages) & 1, kWaitLimitNs)) {
+                            fail();
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int ks = 0; ks < KS; ++ks) {
+                            const int bx = ks / 4, kin = ks % 4;   // box, 32-byte step inside it
+                            const uint64_t adesc = sw128_desc(ksm + bx * kBoxBytes) + uint64_t(kin * 2);
+                            const uint64_t bdesc =
+                                sw128_desc(qsm + st * kQBytes + bx * kBoxBytes) + uint64_t(kin * 2);
+                            tc_mma(d_tmem, adesc, bdesc, kIdesc, (term | ks) != 0 ? 1u : 0u);
+                        }
+                        tc_commit(&qempty[st]);   // stage free once these MMAs are done
+                    }
+                    if (ok) tc_commit(&accfull[acc]);
+                }
+                if (ok) tc_commit(kempty);
+            }
+            // every MMA issued so far has completed before TMEM is released
+            tc_commit(done);
+            if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) fail();
+        }
+    } else {
+        // ------------------------------------------------ epilogue (128 threads)
+        const int quad = warp & 3;              // TMEM lane quadrant of this warp
+        const int row = quad * 32 + lane;       // token row in the tile
+        uint32_t an = 0;
+        for (int64_t it = blockIdx.x; it < ta.items; it += gridDim.x) {
+            const int64_t bh = it / ta.ntiles;
+            const int tile = int(it % ta.ntiles);
+            float tokmax = -INFINITY;
+            bool ok = true;
+            for (int qt = 0; qt < ta.nqt; ++qt, ++an) {
+                const int acc = int(an & 1);
+                const bool got = !aborted() &&
+                                 mbar_wait_bounded(&accfull[acc], (an >> 1) & 1, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) fail();
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * kTileN);
+#pragma unroll
+                for (int ch = 0; ch < kTileN / 32; ++ch) {
+                    float v[32];
+                    tmem_ld32(taddr + uint32_t(ch * 32), v);
+                    const int c0 = qt * kTileN + ch * 32;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (c0 + j < geo.C) tokmax = fmaxf(tokmax, v[j]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[acc]);
+            }
+            if (!ok) break;
+            // span max: S divides 32, tiles start on span boundaries
+            const int64_t moff = int64_t(tile) * kTileM + row;
+            float val = moff < geo.M ? tokmax : -INFINITY;
+            for (int o = 1; o < geo.S; o <<= 1) val = fmaxf(val, __shfl_xor_sync(0xffffffffu, val, o));
+            if (moff < geo.M && (lane % geo.S) == 0) scores[bh * geo.NS + moff / geo.S] = val;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// bf16 terms of the summed group query: [BH][NT][cpad][D]; rows c >= C are 0.
+template <typename T, int D>
+__global__ void qterms_kernel(Geom geo, const T *__restrict__ q, __nv_bfloat16 *__restrict__ out,
+                              int nterms, int cpad)
+{
+    const int64_t total = int64_t(geo.B) * geo.Hkv * nterms * cpad * D;
+    for (int64_t x = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; x < total;
+         x += int64_t(gridDim.x) * blockDim.x) {
+        const int i = int(x % D);
+        const int64_t row = x / D;
+        const int c = int(row % cpad);
+        const int64_t bt = row / cpad;
+        const int term = int(bt % nterms);
+        const int64_t bh = bt / nterms;
+        const int64_t b = bh / geo.Hkv, h = bh % geo.Hkv;
+        float v = 0.f;
+        if (c < geo.C) {
+            if (nterms == geo.g) {   // the group's raw heads: exact products
+                v = Elem<T>::one(q, ((b * geo.Hq + h * geo.g + term) * geo.C + c) * D + i);
+            } else {                 // fp32 sum split into hi + lo
+                float s = 0.f;
+                for (int j = 0; j < geo.g; ++j)
+                    s += Elem<T>::one(q, ((b * geo.Hq + h * geo.g + j) * geo.C + c) * D + i);
+                const float hi = __bfloat162float(__float2bfloat16_rn(s));
+                v = term == 0 ? hi : s - hi;
+            }
+        }
+        out[x] = __float2bfloat16_rn(v);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 map over `rows` rows of D elements, boxes of 128 rows x 64 elements.
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int D)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(D) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_tc_eligible(const Geom &geo)
+{
+    // bf16 inputs, a chunk of queries, spans that tile a 32-token warp
+    return geo.dtype == REATT_BF16 && geo.C > 1 && (32 % geo.S) == 0 &&
+           int64_t(geo.B) * geo.Hkv * geo.T < (int64_t(1) << 31);
+}
+
+static int tc_terms(const Geom &geo) { return geo.g <= 2 ? geo.g : 2; }
+
+size_t prefill_tc_ws_bytes(const Geom &geo)
+{
+    if (!prefill_tc_eligible(geo)) return 0;
+    const int cpad = (geo.C + kTileN - 1) / kTileN * kTileN;
+    return size_t(geo.B) * geo.Hkv * tc_terms(geo) * cpad * geo.d * sizeof(__nv_bfloat16);
+}
+
+cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, float *scores,
+                              void *ws, void *scratch, cudaStream_t st)
+{
+    TcArgs ta;
+    ta.ntiles = int((geo.M + kTileM - 1) / kTileM);
+    ta.items = int64_t(geo.B) * geo.Hkv * ta.ntiles;
+    ta.nqt = (geo.C + kTileN - 1) / kTileN;
+    ta.cpad = ta.nqt * kTileN;
+    ta.nterms = tc_terms(geo);
+    if (ta.items == 0) return cudaSuccess;
+    __nv_bfloat16 *terms = static_cast<__nv_bfloat16 *>(scratch);
+    const int64_t n = int64_t(geo.B) * geo.Hkv * ta.nterms * ta.cpad * geo.d;
+    const int blocks = int((n + 255) / 256 < 8192 ? (n + 255) / 256 : 8192);
+    if (geo.d == 128)
+        qterms_kernel<uint16_t, 128><<<blocks, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q),
+                                                             terms, ta.nterms, ta.cpad);
+    else
+        qterms_kernel<uint16_t, 64><<<blocks, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q),
+                                                            terms, ta.nterms, ta.cpad);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    CUtensorMap kmap, qmap;
+    if (!make_map(&kmap, kc, uint64_t(geo.B) * geo.Hkv * geo.T, geo.d) ||
+        !make_map(&qmap, terms, uint64_t(geo.B) * geo.Hkv * ta.nterms * ta.cpad, geo.d))
+        return cudaErrorInvalidValue;
+    int grid = num_sms();
+    if (ta.items < grid) grid = int(ta.items);
+    const size_t box = kBoxBytes;
+    const size_t smem = 1024 + (geo.d / 64) * box * (1 + kQStages) + (2 + 2 * kQStages + 5) * 8 + 16;
+    if (geo.d == 128) {
+        auto kern = scan_prefill_tc_kernel<128>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kTcThreads, smem, st>>>(kmap, qmap, geo, ta, scores, ws);
+    } else {
+        auto kern = scan_prefill_tc_kernel<64>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kTcThreads, smem, st>>>(kmap, qmap, geo, ta, scores, ws);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace reatt

@@ -317,6 +317,8 @@ topk_slice_kernel(Geom geo, const float *__restrict__ scores, int32_t *__restric
 {
     __shared__ RegScratch rs;
     const int BH = geo.B * geo.Hkv;
+    pdl_wait();      // scores come from the preceding scan
+    pdl_trigger();   // the attention may launch and wait in turn
     if (int(blockIdx.y) >= BH) {   // spare CTA: a chunk of the RoPE table
         fill_rope_table(geo, rope_tab, int64_t(blockIdx.y - BH) * nslices + blockIdx.x);
         return;
@@ -367,6 +369,8 @@ __global__ void __launch_bounds__(kTopkThreads)
 topk_merge_kernel(Geom geo, const uint32_t *__restrict__ cand_code,
                   const int32_t *__restrict__ cand_idx, int32_t *__restrict__ sel, int ncand)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t bh = blockIdx.x;
     const uint32_t *gc = cand_code + bh * int64_t(ncand);
     const int32_t *gi = cand_idx + bh * int64_t(ncand);
@@ -433,10 +437,15 @@ cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void
         tab_rows = (chunks + p.nslices - 1) / p.nslices;
     }
     dim3 grid(unsigned(p.nslices), unsigned(BH + tab_rows));
-    topk_slice_kernel<<<grid, kTopkThreads, 0, st>>>(geo, scores, sel, cc, ci, p.nslices, p.kkp,
-                                                     zero_words, nzero, rope_tab);
-    if (p.nslices > 1 && geo.k > 0)
-        topk_merge_kernel<<<BH, kTopkThreads, 0, st>>>(geo, cc, ci, sel, p.nslices * p.kkp);
+    cudaError_t e = launch_pdl(topk_slice_kernel, grid, dim3(kTopkThreads), 0, st, geo, scores, sel,
+                               cc, ci, p.nslices, p.kkp, zero_words, nzero, rope_tab);
+    if (e != cudaSuccess) return e;
+    if (p.nslices > 1 && geo.k > 0) {
+        e = launch_pdl(topk_merge_kernel, dim3(BH), dim3(kTopkThreads), 0, st, geo,
+                       static_cast<const uint32_t *>(cc), static_cast<const int32_t *>(ci), sel,
+                       p.nslices * p.kkp);
+        if (e != cudaSuccess) return e;
+    }
     return cudaGetLastError();
 }
 
