@@ -171,6 +171,34 @@ REATT_API int reatt_step(const reatt_dims *dims, const void *q, const void *k_ca
                const void *k_cur, const void *v_cur, int32_t *sel_out, float *out, void *ws,
                reatt_stream stream);
 
+/*
+ * reatt_step without a caller-supplied workspace.  The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory: a plugin interface that gives its kernels no allocator, or a
+ * latency-critical loop where cudaMalloc would synchronize the device.
+ *
+ * Same arguments, results and errors as reatt_step, minus `ws`.  The
+ * workspace is a 16 MiB (16 * 2^20 bytes) array in the library's device
+ * globals, which every GPU that loads the library holds until the process
+ * exits.  Calls whose reatt_workspace_bytes() exceeds 16 MiB return
+ * REATT_EUNSUPPORTED before anything is launched.  For scale: the 128K
+ * LLaMA3-8B-shaped decode needs 3.4 MiB, the 4M-token Qwen2-1.5B-shaped decode
+ * 4.4 MiB, four 1M-token LLaMA3-8B-shaped sequences 7.5 MiB, and a 2048-query
+ * prefill chunk over 256K tokens 12.3 MiB.
+ *   - Allocates nothing: no cudaMalloc/cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, which also loads the library's device globals
+ *     there); make that first call before any stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents; what must start at zero is cleared inside each call.  Calls
+ *     that overlap on the GPU race: order them on one stream.
+ *   - A bounded-wait timeout is recorded in the shared array's status word,
+ *     which this call does not expose.
+ */
+REATT_API int reatt_step_fixed_scratch(const reatt_dims *dims, const void *q, const void *k_cache,
+                                       const void *v_cache, const void *k_cur, const void *v_cur,
+                                       int32_t *sel_out, float *out, reatt_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,7 +20,7 @@ F32, BF16 = 0, 1
 
 EXPORTS = ["reatt_status_string", "reatt_num_spans", "reatt_window_max", "reatt_workspace_bytes",
            "reatt_workspace_status", "reatt_score_spans", "reatt_topk", "reatt_gather_rope",
-           "reatt_attend", "reatt_step"]
+           "reatt_attend", "reatt_step", "reatt_step_fixed_scratch"]
 
 
 class reatt_dims(ctypes.Structure):
@@ -53,6 +53,7 @@ lib.reatt_topk.argtypes = [_dp, _vp, _vp, _vp, _vp]
 lib.reatt_gather_rope.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.reatt_attend.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.reatt_step.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.reatt_step_fixed_scratch.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 for _name in EXPORTS[1:]:
     getattr(lib, _name).restype = ctypes.c_int
 
@@ -165,6 +166,18 @@ def reatt_step(dims, q, k_cache, v_cache, k_cur, v_cur, sel_out, out, ws, stream
                         _ptr(v_cur), _ptr(sel_out), _ptr(out), _ptr(ws), _stream(stream))
     if check:
         _check(rc, "reatt_step")
+    return rc
+
+
+def reatt_step_fixed_scratch(dims, q, k_cache, v_cache, k_cur, v_cur, sel_out, out, stream=None,
+                             check=True):
+    """reatt_step with the library's fixed 16 MiB device scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    rc = lib.reatt_step_fixed_scratch(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(k_cur), _ptr(v_cur), _ptr(sel_out), _ptr(out),
+                                      _stream(stream))
+    if check:
+        _check(rc, "reatt_step_fixed_scratch")
     return rc
 
 
