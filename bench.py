@@ -125,6 +125,16 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def aggregate(world, step_b, steps, total_ms, e2e_ms, scan_ms, reduce_max=None):
+    """Whole-job numbers: the slowest rank's times (max over ranks) and the
+    bytes of every rank's replica over that time (weak scaling)."""
+    if world > 1:
+        total_ms, e2e_ms, scan_ms = reduce_max([total_ms, e2e_ms, scan_ms])
+    return {"total_ms": total_ms, "e2e_ms": e2e_ms, "scan_ms": scan_ms,
+            "value": world * step_b * steps / (total_ms * 1e-3) / 1e9,
+            "e2e_value": world * step_b * steps / (e2e_ms * 1e-3) / 1e9}
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -252,15 +262,17 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
 
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms, scan_ms], dtype=torch.float64, device=dev)
+    def reduce_max(vals):
+        t = torch.tensor(vals, dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms, scan_ms = (float(v) for v in t.tolist())
+        return [float(v) for v in t.tolist()]
 
     scan_b, step_b = step_bytes(w)
+    agg = aggregate(world, step_b, args.steps, total_ms, e2e_ms, scan_ms,
+                    reduce_max if world > 1 else None)
+    total_ms, e2e_ms, scan_ms = agg["total_ms"], agg["e2e_ms"], agg["scan_ms"]
     ms_per_step = total_ms / args.steps
-    value = world * step_b * args.steps / (total_ms * 1e-3) / 1e9
-    e2e_value = world * step_b * args.steps / (e2e_ms * 1e-3) / 1e9
+    value, e2e_value = agg["value"], agg["e2e_value"]
     peak, peak_kind = peaks()
     achieved = scan_b / (scan_ms * 1e-3) / 1e9
     result = {
