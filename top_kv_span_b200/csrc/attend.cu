@@ -574,16 +574,18 @@ attend_decode_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
 // (cp.async.bulk, mbarrier completion).  Consumer warp w takes chunks w,
 // w+NCW, ... (fixed stage -> warp map, so parity waits never run ahead) and
 // computes as the register kernel above, reading its pair words from shared
-// memory.  RoPE cos/sin come from the fp32 reduced angle at the start of each
-// sub-batch, advanced key by key with the constant one-position rotation.
-constexpr int kTmaCW = 16;                 // consumer warps
-constexpr int kTmaStages = 16;             // multiple of kTmaCW
+// memory.  The step's RoPE cos/sin table rows for the chunk's positions come
+// into the same ring stage.
+constexpr int kTmaCW = 12;                 // consumer warps (13 warps: <= 128 registers)
+constexpr int kTmaStages = 2 * kTmaCW;     // warp w owns stages w and w + kTmaCW
 
-template <typename T, int D>
+template <typename T, int D, int RP>
 struct TmaShape {
     static constexpr int kRowBytes = D * Elem<T>::kBytes;
-    static constexpr int kChunk = kRowBytes >= 512 ? 8 : 16;          // rows per ring stage
-    static constexpr int kStageBytes = 2 * kChunk * kRowBytes;         // K rows then V rows
+    static constexpr int kTabRowBytes = D / 2 * 8;                     // (cos, sin) per pair
+    static constexpr int kChunk = (RP <= 4 && kRowBytes <= 256) ? 8 : 4;   // rows per stage
+    // K rows, then V rows, then the rows' RoPE table entries
+    static constexpr int kStageBytes = kChunk * (2 * kRowBytes + kTabRowBytes);
     static constexpr size_t kRing = size_t(kTmaStages) * kStageBytes;
 };
 static_assert(kTmaStages % kTmaCW == 0, "stage -> warp map must be fixed");
@@ -619,13 +621,13 @@ __global__ void __launch_bounds__((kTmaCW + 1) * 32, 1)
 attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__restrict__ vc,
                      const T *__restrict__ kcur, const T *__restrict__ vcur, void *ws)
 {
-    using Sh = TmaShape<T, D>;
+    using Sh = TmaShape<T, D, RP>;
     constexpr int PD = D / 64;            // RoPE pairs per lane
     constexpr int KB = 32 / RP;           // keys per reduction batch
     constexpr int RB = Sh::kRowBytes;
     constexpr int CH = Sh::kChunk;
     constexpr int EB = Elem<T>::kBytes;
-    static_assert(kTmaStages == kTmaCW, "warp w owns ring stage w");
+    static_assert(kTmaStages % kTmaCW == 0, "chunk ci -> stage ci % kTmaStages -> warp ci % kTmaCW");
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *ring = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Sh::kRing);
@@ -687,17 +689,19 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
 
     const int nchunks = kend > kbeg ? (kend - kbeg + CH - 1) / CH : 0;
     if (warp == kTmaCW) {
-        // ------------------------------------------------ producer (one thread)
+        // ------------------------------------------------ producer warp
         // chunk ci = window rows [kbeg + ci*CH, +CH) -> stage ci % kTmaStages;
-        // a chunk crossing a region boundary is copied as several runs
-        if (lane == 0) {
+        // lane l issues every chunk of stage l, in order, so each barrier has
+        // one waiter taking its phases in turn.  A chunk crossing a region
+        // boundary is copied as several runs.
+        static_assert(kTmaStages <= 32, "one producer lane per stage");
+        if (lane < kTmaStages) {
             int issued = 0;
-            for (int ci = 0; ci < nchunks; ++ci, ++issued) {
-                const int stage = ci % kTmaStages;
-                if (ci >= kTmaStages &&
+            for (int ci = lane; ci < nchunks; ci += kTmaStages, ++issued) {
+                const int stage = lane;
+                if (issued > 0 &&
                     (*(volatile int *)&abort_flag ||
-                     !mbar_wait_bounded(&empty[stage], uint32_t(((ci / kTmaStages) - 1) & 1),
-                                        kWaitLimitNs))) {
+                     !mbar_wait_bounded(&empty[stage], uint32_t((issued - 1) & 1), kWaitLimitNs))) {
                     report_status(ws, REATT_ETIMEOUT);
                     *(volatile int *)&abort_flag = 1;
                     break;
@@ -705,7 +709,9 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
                 const int p0 = kbeg + ci * CH;
                 const int n = kend - p0 < CH ? kend - p0 : CH;
                 uint8_t *dst = ring + stage * Sh::kStageBytes;
-                mbar_arrive_expect_tx(&full[stage], 2u * uint32_t(n) * RB);
+                mbar_arrive_expect_tx(&full[stage], uint32_t(n) * (2u * RB + Sh::kTabRowBytes));
+                bulk_load_plain(dst + 2 * CH * RB, a.tab + int64_t(p0) * (D / 2),
+                                uint32_t(n) * Sh::kTabRowBytes, &full[stage]);
                 for (int p = p0; p < p0 + n;) {
                     const int r = chunk_len(geo, m, p, p0 + n, CH);
                     bool cur = false;
@@ -732,20 +738,16 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
                     p += r;
                 }
             }
-            // drain: the last use of every stage that was issued
-            for (int ci = issued - 1; ci >= 0 && ci >= issued - kTmaStages; --ci)
-                if (!mbar_wait_bounded(&full[ci % kTmaStages], uint32_t((ci / kTmaStages) & 1),
-                                       kWaitLimitNs))
-                    report_status(ws, REATT_ETIMEOUT);
+            // drain: this stage's last issued copy has landed
+            if (issued > 0 && !mbar_wait_bounded(&full[lane], uint32_t((issued - 1) & 1), kWaitLimitNs))
+                report_status(ws, REATT_ETIMEOUT);
         }
     } else {
         // ---------------------------------------------------- consumers
         float qlo[RP][PD], qhi[RP][PD];
-        float2 step[PD];   // (cos, sin) of one position step, per pair
 #pragma unroll
         for (int e = 0; e < PD; ++e) {
             const int i = PD * lane + e;
-            rope_cs(1, freq[i].x, freq[i].y, step[e].x, step[e].y);
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 qlo[r][e] = q_s[r][i];
@@ -780,12 +782,7 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
             }
             const uint8_t *kb = ring + stage * Sh::kStageBytes;
             const uint8_t *vb = kb + CH * RB;
-            float2 cs[PD];   // RoPE of this lane's pairs at the chunk's first row
-#pragma unroll
-            for (int e = 0; e < PD; ++e) {
-                const int i = PD * lane + e;
-                rope_cs(p0, freq[i].x, freq[i].y, cs[e].x, cs[e].y);
-            }
+            const float2 *tb = reinterpret_cast<const float2 *>(kb + 2 * CH * RB);
             for (int sb = 0; sb < n; sb += KB) {
                 float part[32];
 #pragma unroll
@@ -802,14 +799,14 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
 #pragma unroll
                         for (int e = 0; e < PD; ++e) klo[e] = khi[e] = 0.f;
                     }
+                    if (row < n) {   // rotate at window position p0 + row
 #pragma unroll
-                    for (int e = 0; e < PD; ++e) {
-                        const float x0 = klo[e], x1 = khi[e];
-                        klo[e] = x0 * cs[e].x - x1 * cs[e].y;
-                        khi[e] = x1 * cs[e].x + x0 * cs[e].y;
-                        const float c2 = cs[e].x * step[e].x - cs[e].y * step[e].y;
-                        cs[e].y = cs[e].y * step[e].x + cs[e].x * step[e].y;
-                        cs[e].x = c2;
+                        for (int e = 0; e < PD; ++e) {
+                            const float2 cs = tb[row * (D / 2) + PD * lane + e];
+                            const float x0 = klo[e], x1 = khi[e];
+                            klo[e] = x0 * cs.x - x1 * cs.y;
+                            khi[e] = x1 * cs.x + x0 * cs.y;
+                        }
                     }
 #pragma unroll
                     for (int r = 0; r < RP; ++r) {
@@ -927,12 +924,12 @@ cudaError_t launch_staged_attn(const Geom &geo, const AttnArgs &a, int RP, const
                                const void *vc, const void *kcur, const void *vcur, void *ws,
                                cudaStream_t st)
 {
-    using Sh = TmaShape<T, D>;
     dim3 grid(unsigned(a.nsplit), 1u, unsigned(geo.B * geo.Hkv));
     const T *k = static_cast<const T *>(kc), *v = static_cast<const T *>(vc);
     const T *kq = static_cast<const T *>(kcur), *vq = static_cast<const T *>(vcur);
 #define REATT_STAGED(RPV)                                                                      \
     do {                                                                                       \
+        using Sh = TmaShape<T, D, RPV>;                                                        \
         const size_t smem = Sh::kRing + 2 * kTmaStages * sizeof(uint64_t) +                   \
                             size_t(kTmaCW) * RPV * (D + 2) * sizeof(float);                    \
         auto kern = attend_staged_kernel<T, D, RPV>;                                           \
