@@ -1279,7 +1279,8 @@ AttnPlan attn_plan(const Geom &geo)
         p.decode = true;
         p.QB = R <= 1 ? 1 : R <= 2 ? 2 : R <= 4 ? 4 : 8;
         p.nqb = 1;
-        int64_t ns = (kDecodeCtas + BH - 1) / BH;
+        // one wave: the staged kernel holds one CTA per SM
+        int64_t ns = kDecodeCtas / BH;
         const int64_t max_split = (geo.Wmax + kMinSplitKeys - 1) / kMinSplitKeys;
         const int64_t cap = int64_t(kDecWarps - 1) * geo.d;   // combine scratch (floats / QB)
         if (ns > max_split) ns = max_split;
