@@ -183,8 +183,9 @@ REATT_API int reatt_step(const reatt_dims *dims, const void *q, const void *k_ca
  * exits.  Calls whose reatt_workspace_bytes() exceeds 16 MiB return
  * REATT_EUNSUPPORTED before anything is launched.  For scale: the 128K
  * LLaMA3-8B-shaped decode needs 3.4 MiB, the 4M-token Qwen2-1.5B-shaped decode
- * 4.4 MiB, four 1M-token LLaMA3-8B-shaped sequences 7.5 MiB, and a 2048-query
- * prefill chunk over 256K tokens 12.3 MiB.
+ * 4.4 MiB, four 1M-token LLaMA3-8B-shaped sequences 7.4 MiB; a 2048-query
+ * bf16 prefill chunk over 256K tokens needs 92.7 MiB (its tensor-core
+ * attention operands) and is rejected.
  *   - Allocates nothing: no cudaMalloc/cudaFree or allocating library call.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, which also loads the library's device globals

@@ -64,9 +64,10 @@ int make_geom(const reatt_dims *d, Geom *g)
 }
 
 // Workspace layout: [status header][attention tickets][attention partials]
-// [top-k candidates][summed queries (C > 1)][span scores][selection][RoPE table].
+// [top-k candidates][summed queries (C > 1)][span scores][selection][RoPE table]
+// [prefill attention operands].
 struct WsPlan {
-    size_t ticket, ticket_bytes, topk, qsum, scores, sel, tab, total;
+    size_t ticket, ticket_bytes, topk, qsum, scores, sel, tab, fa, total;
 };
 WsPlan ws_plan(const Geom &g)
 {
@@ -87,6 +88,8 @@ WsPlan ws_plan(const Geom &g)
     off = up256(off + size_t(g.B) * g.Hkv * g.k * sizeof(int32_t));
     p.tab = off;
     off = up256(off + rope_table_bytes(g));
+    p.fa = off;
+    off = up256(off + prefill_attn_tc_ws_bytes(g));
     p.total = off;
     return p;
 }
@@ -249,6 +252,9 @@ int reatt_step(const reatt_dims *dims, const void *q, const void *k_cache, const
     e = launch_topk(g, scores, sel, at(ws, p.topk), reinterpret_cast<uint32_t *>(at(ws, p.ticket)),
                     int(p.ticket_bytes / sizeof(uint32_t)), tab, st);
     if (e != cudaSuccess) return REATT_ECUDA;
+    if (prefill_attn_tc_eligible(g))   // many query rows: tensor-core attention
+        return cuda_status(launch_attend_prefill_tc(g, q, k_cache, v_cache, k_cur, v_cur, sel, tab,
+                                                    out, at(ws, p.fa), ws, st));
     return cuda_status(launch_attend(g, q, nullptr, nullptr, nullptr, k_cache, v_cache, k_cur,
                                      v_cur, sel, tab, out, at(ws, p.ticket), ws, true, st));
 }

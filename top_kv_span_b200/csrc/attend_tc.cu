@@ -1,0 +1,608 @@
+// Chunked-prefill attention over the window on the tensor cores (tcgen05 + TMEM).
+//
+// The window of one (batch, KV head) and the chunk's g*C query rows form a
+// causal attention (ReAttention OpenReview discussion, "Prefilling Phase":
+// flash_attention(query, key_recall, value_recall); research-map summary
+// "Approach": RoPE applied after concatenation, window row p at position p,
+// query c at W-C+c).  To keep fp32-level accuracy with bf16 tensor-core
+// operands every rotated operand is split into bf16 hi + lo:
+//   S = Qh.Kh^T + Qh.Kl^T + Ql.Kh^T   (dropped Ql.Kl^T is ~2^-18 relative)
+//   O += Ph.V + Pl.V                  (V is exact: bf16 input)
+//
+// prefill_prep_kernel writes, per KV head, the rotated+scaled query rows
+// (hi/lo), the rotated window keys (hi/lo) and the window values transposed,
+// all bf16, from the un-rotated cache through the selection (the window is
+// never materialised in fp32).  attend_prefill_tc_kernel then runs, per
+// 128-row query block:
+//   warp 0   TMA producer: the query block once, then 64-key tiles of K (hi,
+//            lo) and V^T in a 2-stage ring (128B swizzle, no multicast)
+//   warp 1   TMEM allocation; one thread issues S(j) into one of two TMEM
+//            S buffers, then O += P(j-1).V(j-1) into the TMEM O accumulator
+//   warps 2-5 softmax: one thread per query row reads its S row from TMEM,
+//            masks (causal, window end), keeps a running reference max that
+//            moves (and rescales O in TMEM) only when the row max grows by
+//            more than 2^8, writes P as bf16 hi/lo in the swizzled operand
+//            layout, and finally divides O by the row sum.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace reatt {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kFaThreads = 6 * 32;
+constexpr int kQRows = 128;   // query rows per CTA (TMEM lanes)
+constexpr int kKeyTile = 64;  // keys per S tile (S columns)
+constexpr float kRescaleLog2 = 8.f;
+
+struct WinMapTc {
+    int64_t g_end, loc_begin, n_loc, nsel_rows, W;
+};
+
+__device__ __forceinline__ WinMapTc winmap_tc(const Geom &geo, const int32_t *sel_bh)
+{
+    WinMapTc m;
+    m.g_end = geo.g_end;
+    m.loc_begin = geo.loc_begin;
+    m.n_loc = geo.n_loc;
+    const int64_t keff = geo.k < geo.NS ? geo.k : geo.NS;
+    m.nsel_rows = keff * geo.S;
+    if (keff > 0) {
+        const int32_t last = sel_bh[keff - 1];
+        const int64_t r = geo.M % geo.S;
+        if (last == geo.NS - 1 && r != 0) m.nsel_rows -= geo.S - r;
+    }
+    m.W = m.g_end + m.nsel_rows + m.n_loc + geo.C;
+    return m;
+}
+
+// Window row p -> element offset of its K/V row (bit 62: current token).
+__device__ __forceinline__ int64_t row_src_tc(const Geom &geo, const WinMapTc &m,
+                                              const int32_t *sel_bh, int64_t bh, int64_t p, int D)
+{
+    if (p < m.g_end) return (bh * geo.T + p) * D;
+    p -= m.g_end;
+    if (p < m.nsel_rows) {
+        const int64_t j = p / geo.S, off = p - j * geo.S;
+        int64_t sp = sel_bh[j];
+        sp = sp < 0 ? 0 : (sp >= geo.NS ? geo.NS - 1 : sp);
+        int64_t row = geo.G + sp * geo.S + off;
+        if (row >= geo.T) row = geo.T - 1;
+        return (bh * geo.T + row) * D;
+    }
+    p -= m.nsel_rows;
+    if (p < m.n_loc) return (bh * geo.T + m.loc_begin + p) * D;
+    return (int64_t(1) << 62) | ((bh * geo.C + (p - m.n_loc)) * D);
+}
+
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo)
+{
+    hi = __float2bfloat16_rn(x);
+    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
+// Operand buffers of one call, bf16, per KV head bh:
+//   qh/ql [BH][Rp][D]  rotated queries x log2(e)/sqrt(d), rows >= R zero
+//   kh/kl [BH][Wp][D]  rotated window keys, rows >= W zero
+//   vt    [BH][D][Wp]  window values transposed, columns >= W zero
+struct PrepOut {
+    __nv_bfloat16 *qh, *ql, *kh, *kl, *vt;
+    int Rp, Wp;
+};
+
+constexpr int kPrepRows = 64;
+
+template <int D>
+__global__ void __launch_bounds__(256)
+prefill_prep_kernel(Geom geo, const uint16_t *__restrict__ q, const uint16_t *__restrict__ kc,
+                    const uint16_t *__restrict__ vc, const uint16_t *__restrict__ kcur,
+                    const uint16_t *__restrict__ vcur, const int32_t *__restrict__ sel,
+                    const float2 *__restrict__ tab, PrepOut po)
+{
+    __shared__ float vs[kPrepRows][D + 1];
+    __shared__ float2 freq[D / 2];
+    pdl_wait();   // the selection and the RoPE table come from the top-k launch
+    const int64_t bh = blockIdx.y;
+    const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv);
+    const int32_t *sel_bh = sel + bh * geo.k;
+    const WinMapTc m = winmap_tc(geo, sel_bh);
+    if (threadIdx.x < D / 2) freq[threadIdx.x] = make_float2(geo.rope_hi[threadIdx.x], geo.rope_lo[threadIdx.x]);
+    __syncthreads();
+    const int nkb = po.Wp / kPrepRows;
+    if (int(blockIdx.x) < nkb) {
+        // ---- 64 window rows: rotated K hi/lo, V transposed
+        const int64_t p0 = int64_t(blockIdx.x) * kPrepRows;
+        for (int x = threadIdx.x; x < kPrepRows * (D / 2); x += blockDim.x) {
+            const int r = x / (D / 2), i = x % (D / 2);
+            const int64_t p = p0 + r;
+            float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+            if (p < m.W) {
+                const int64_t off = row_src_tc(geo, m, sel_bh, bh, p, D);
+                const bool cur = (off >> 62) != 0;
+                const int64_t o = off & ~(int64_t(1) << 62);
+                const uint16_t *kr = (cur ? kcur : kc) + o, *vr = (cur ? vcur : vc) + o;
+                const float a = Elem<uint16_t>::one(kr, i), c = Elem<uint16_t>::one(kr, i + D / 2);
+                const float2 cs = tab[p * (D / 2) + i];
+                k0 = a * cs.x - c * cs.y;
+                k1 = c * cs.x + a * cs.y;
+                v0 = Elem<uint16_t>::one(vr, i);
+                v1 = Elem<uint16_t>::one(vr, i + D / 2);
+            }
+            const int64_t kb = (bh * po.Wp + p) * D;
+            split_bf16(k0, po.kh[kb + i], po.kl[kb + i]);
+            split_bf16(k1, po.kh[kb + i + D / 2], po.kl[kb + i + D / 2]);
+            vs[r][i] = v0;
+            vs[r][i + D / 2] = v1;
+        }
+        __syncthreads();
+        for (int x = threadIdx.x; x < D * kPrepRows; x += blockDim.x) {
+            const int i = x / kPrepRows, r = x % kPrepRows;
+            po.vt[(bh * D + i) * po.Wp + p0 + r] = __float2bfloat16_rn(vs[r][i]);
+        }
+    } else {
+        // ---- 64 query rows: rotated at W-C+c, scaled, hi/lo
+        const int64_t r0 = int64_t(int(blockIdx.x) - nkb) * kPrepRows;
+        const int R = geo.g * geo.C;
+        const float qscale = 1.4426950408889634f * rsqrtf(float(D));
+        const int64_t qpos0 = m.W - geo.C;
+        for (int x = threadIdx.x; x < kPrepRows * (D / 2); x += blockDim.x) {
+            const int rr = x / (D / 2), i = x % (D / 2);
+            const int64_t r = r0 + rr;
+            float lo = 0.f, hi = 0.f;
+            if (r < R) {
+                const int j = h * geo.g + int(r / geo.C), c = int(r % geo.C);
+                const uint16_t *qr = q + ((int64_t(b) * geo.Hq + j) * geo.C + c) * D;
+                const float x0 = Elem<uint16_t>::one(qr, i), x1 = Elem<uint16_t>::one(qr, i + D / 2);
+                float cs, sn;
+                rope_cs(qpos0 + c, freq[i].x, freq[i].y, cs, sn);
+                lo = (x0 * cs - x1 * sn) * qscale;
+                hi = (x1 * cs + x0 * sn) * qscale;
+            }
+            const int64_t qb = (bh * po.Rp + r) * D;
+            split_bf16(lo, po.qh[qb + i], po.ql[qb + i]);
+            split_bf16(hi, po.qh[qb + i + D / 2], po.ql[qb + i + D / 2]);
+        }
+    }
+}
+
+struct FaArgs {
+    float *out;
+    const int32_t *sel;
+    int Rp, Wp;
+};
+
+// Shared-memory plan (1024-byte aligned): Qh | Ql | K stage 0,1 (hi | lo) |
+// V^T stage 0,1 | Ph | Pl | barriers.
+template <int D>
+struct FaSmem {
+    static constexpr int NBOX = D / 64;
+    static constexpr int kQ = NBOX * kQRows * 128;       // one of Qh / Ql
+    static constexpr int kK = NBOX * kKeyTile * 128;     // one of Kh / Kl
+    static constexpr int kV = D * kKeyTile * 2;          // V^T tile: D rows x 64 keys
+    static constexpr int kP = kQRows * kKeyTile * 2;     // one of Ph / Pl
+    static constexpr int oQh = 0, oQl = kQ, oK = 2 * kQ, oV = oK + 4 * kK, oP = oV + 2 * kV,
+                         oBar = oP + 2 * kP;
+    static constexpr size_t kBytes = size_t(oBar) + 32 * 8 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kFaThreads, 1)
+attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
+                         const __grid_constant__ CUtensorMap qlmap,
+                         const __grid_constant__ CUtensorMap khmap,
+                         const __grid_constant__ CUtensorMap klmap,
+                         const __grid_constant__ CUtensorMap vtmap, Geom geo, FaArgs fa, void *ws)
+{
+    using Sm = FaSmem<D>;
+    constexpr int NBOX = Sm::NBOX;
+    constexpr int KS = D / 16;                 // k-steps of S over the head width
+    constexpr int PS = kKeyTile / 16;          // k-steps of P.V over a key tile
+    constexpr uint32_t kTmemCols = 256;        // S buffers at 0 and 64, O at 128
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Sm::oBar);
+    uint64_t *qfull = bars, *kfull = bars + 1, *kempty = bars + 3, *vfull = bars + 5,
+             *vempty = bars + 7, *sfull = bars + 9, *sempty = bars + 11, *pfull = bars + 13,
+             *pvdone = bars + 14, *done = bars + 15;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    __shared__ int abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        abort_flag = 0;
+        mbar_init(qfull, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&kfull[s], 1);
+            mbar_init(&kempty[s], 1);
+            mbar_init(&vfull[s], 1);
+            mbar_init(&vempty[s], 1);
+            mbar_init(&sfull[s], 1);
+            mbar_init(&sempty[s], 4);
+        }
+        mbar_init(pfull, 4);
+        mbar_init(pvdone, 1);
+        mbar_init(done, 1);
+        mbar_init_fence();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    pdl_wait();   // operands come from the prep launch
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int qb = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv);
+    const int R = geo.g * geo.C;
+    const int r0 = qb * kQRows;
+    const int nrows = R - r0 < kQRows ? R - r0 : kQRows;
+    const WinMapTc m = winmap_tc(geo, fa.sel + bh * geo.k);
+    const int64_t W = m.W, qpos0 = W - geo.C;
+    const int last_row = r0 + nrows - 1;
+    const int c_max = (last_row / geo.C == r0 / geo.C) ? last_row % geo.C : geo.C - 1;
+    int64_t kend = qpos0 + c_max + 1;
+    if (kend > W) kend = W;
+    const int nt = int((kend + kKeyTile - 1) / kKeyTile);
+
+    auto fail = [&]() {
+        report_status(ws, REATT_ETIMEOUT);
+        *(volatile int *)&abort_flag = 1;
+    };
+    auto aborted = [&]() { return *(volatile int *)&abort_flag != 0; };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            const int qy = int(bh * fa.Rp + r0);
+            mbar_arrive_expect_tx(qfull, 2 * Sm::kQ);
+            for (int bx = 0; bx < NBOX; ++bx) {
+                tma_load_2d(smem + Sm::oQh + bx * kQRows * 128, &qhmap, 64 * bx, qy, qfull);
+                tma_load_2d(smem + Sm::oQl + bx * kQRows * 128, &qlmap, 64 * bx, qy, qfull);
+            }
+            for (int j = 0; ok && j < nt; ++j) {
+                const int s = j & 1;
+                if (j >= 2 && (aborted() || !mbar_wait_bounded(&kempty[s], ((j >> 1) - 1) & 1, kWaitLimitNs))) {
+                    fail();
+                    ok = false;
+                    break;
+                }
+                const int ky = int(bh * fa.Wp + int64_t(j) * kKeyTile);
+                uint8_t *kst = smem + Sm::oK + s * 2 * Sm::kK;
+                mbar_arrive_expect_tx(&kfull[s], 2 * Sm::kK);
+                for (int bx = 0; bx < NBOX; ++bx) {
+                    tma_load_2d(kst + bx * kKeyTile * 128, &khmap, 64 * bx, ky, &kfull[s]);
+                    tma_load_2d(kst + Sm::kK + bx * kKeyTile * 128, &klmap, 64 * bx, ky, &kfull[s]);
+                }
+                if (j >= 2 && (aborted() || !mbar_wait_bounded(&vempty[s], ((j >> 1) - 1) & 1, kWaitLimitNs))) {
+                    fail();
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&vfull[s], Sm::kV);
+                tma_load_2d(smem + Sm::oV + s * Sm::kV, &vtmap, j * kKeyTile, int(bh * D), &vfull[s]);
+            }
+            // drain the loads in flight
+            if (!mbar_wait_bounded(qfull, 0, kWaitLimitNs)) fail();
+            for (int j = nt - 2 < 0 ? 0 : nt - 2; j < nt; ++j) {
+                if (!mbar_wait_bounded(&kfull[j & 1], (j >> 1) & 1, kWaitLimitNs)) fail();
+                if (!mbar_wait_bounded(&vfull[j & 1], (j >> 1) & 1, kWaitLimitNs)) fail();
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(kQRows, kKeyTile), id_o = idesc_bf16(kQRows, D);
+            bool ok = !aborted() && mbar_wait_bounded(qfull, 0, kWaitLimitNs);
+            if (!ok) fail();
+            tc_fence_after();
+            for (int j = 0; ok && j <= nt; ++j) {
+                if (j < nt) {   // S(j) = Q.K(j)^T (three hi/lo products)
+                    const int s = j & 1;
+                    if (aborted() || !mbar_wait_bounded(&kfull[s], (j >> 1) & 1, kWaitLimitNs) ||
+                        (j >= 2 && !mbar_wait_bounded(&sempty[s], ((j >> 1) - 1) & 1, kWaitLimitNs))) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t *kst = smem + Sm::oK + s * 2 * Sm::kK;
+                    const uint32_t d_s = tmem_base + uint32_t(s * kKeyTile);
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks) {
+                        const int bx = ks / 4, kin = ks % 4;
+                        const uint64_t qh = sw128_desc(smem + Sm::oQh + bx * kQRows * 128) + uint64_t(kin * 2);
+                        const uint64_t ql = sw128_desc(smem + Sm::oQl + bx * kQRows * 128) + uint64_t(kin * 2);
+                        const uint64_t kh = sw128_desc(kst + bx * kKeyTile * 128) + uint64_t(kin * 2);
+                        const uint64_t kl = sw128_desc(kst + Sm::kK + bx * kKeyTile * 128) + uint64_t(kin * 2);
+                        tc_mma(d_s, qh, kh, id_s, ks > 0 ? 1u : 0u);
+                        tc_mma(d_s, qh, kl, id_s, 1u);
+                        tc_mma(d_s, ql, kh, id_s, 1u);
+                    }
+                    tc_commit(&sfull[s]);
+                    tc_commit(&kempty[s]);
+                }
+                if (j >= 1) {   // O += P(j-1).V(j-1) (hi and lo P)
+                    const int jj = j - 1, s = jj & 1;
+                    if (aborted() || !mbar_wait_bounded(pfull, jj & 1, kWaitLimitNs) ||
+                        !mbar_wait_bounded(&vfull[s], (jj >> 1) & 1, kWaitLimitNs)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_o = tmem_base + 128u;
+                    const uint8_t *vst = smem + Sm::oV + s * Sm::kV;
+#pragma unroll
+                    for (int ks = 0; ks < PS; ++ks) {
+                        const uint64_t ph = sw128_desc(smem + Sm::oP) + uint64_t(ks * 2);
+                        const uint64_t pl = sw128_desc(smem + Sm::oP + Sm::kP) + uint64_t(ks * 2);
+                        const uint64_t vd = sw128_desc(vst) + uint64_t(ks * 2);
+                        tc_mma(d_o, ph, vd, id_o, (jj > 0 || ks > 0) ? 1u : 0u);
+                        tc_mma(d_o, pl, vd, id_o, 1u);
+                    }
+                    tc_commit(pvdone);
+                    tc_commit(&vempty[s]);
+                }
+            }
+            tc_commit(done);
+            if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) fail();
+        }
+    } else {
+        // ------------------------------------------------ softmax warps (one query row each)
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = tmem_base + (uint32_t(quad * 32) << 16);
+        const bool live = row < nrows;
+        const int64_t qpos = live ? qpos0 + (r0 + row) % geo.C : -1;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        uint8_t *ph = smem + Sm::oP, *pl = smem + Sm::oP + Sm::kP;
+        for (int j = 0; j < nt; ++j) {
+            const int s = j & 1;
+            bool got = !aborted() && mbar_wait_bounded(&sfull[s], (j >> 1) & 1, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, got)) {
+                if (lane == 0) fail();
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float sv[kKeyTile];
+            {
+                float t[32];
+                tmem_ld32(lane_base + uint32_t(s * kKeyTile), t);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[i] = t[i];
+                tmem_ld32(lane_base + uint32_t(s * kKeyTile + 32), t);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[32 + i] = t[i];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sempty[s]);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kKeyTile; ++i) {
+                const int64_t kp = int64_t(j) * kKeyTile + i;
+                if (!(kp < kend && kp <= qpos)) sv[i] = -INFINITY;
+                mx = fmaxf(mx, sv[i]);
+            }
+            // the P buffer and O are free once P(j-1).V(j-1) has completed
+            if (j >= 1) {
+                got = !aborted() && mbar_wait_bounded(pvdone, (j - 1) & 1, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) fail();
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            const float m_new = fmaxf(m_ref, mx);
+            const bool move = m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kRescaleLog2);
+            float fac = 1.f;
+            if (move) {
+                fac = m_ref == -INFINITY ? 0.f : exp2f(m_ref - m_new);
+                m_ref = m_new;
+                l *= fac;
+            }
+            if (j >= 1 && __any_sync(0xffffffffu, move && fac != 1.f)) {
+                // rescale this row of O in TMEM (warp-collective accesses)
+#pragma unroll
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    float o[32];
+                    const uint32_t ta = lane_base + 128u + uint32_t(cb * 32);
+                    tmem_ld32(ta, o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] *= fac;
+                    tmem_st32(ta, o);
+                }
+            }
+            // P = exp2(S - m_ref) as bf16 hi + lo, 128B-swizzled K-major rows
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < kKeyTile / 8; ++c) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    float p0 = sv[c * 8 + e] == -INFINITY ? 0.f : exp2f(sv[c * 8 + e] - m_ref);
+                    float p1 = sv[c * 8 + e + 1] == -INFINITY ? 0.f : exp2f(sv[c * 8 + e + 1] - m_ref);
+                    if (!live) p0 = p1 = 0.f;
+                    rs += p0 + p1;
+                    const __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+                    const float2 hf = __bfloat1622float2(hv);
+                    const __nv_bfloat162 lv = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                    hw[e / 2] = *reinterpret_cast<const uint32_t *>(&hv);
+                    lw[e / 2] = *reinterpret_cast<const uint32_t *>(&lv);
+                }
+                const int phys = (c ^ (row & 7)) * 16;
+                *reinterpret_cast<uint4 *>(ph + row * 128 + phys) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(pl + row * 128 + phys) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            l += rs;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pfull);
+        }
+        if (ok && nt > 0) {
+            const bool got = !aborted() && mbar_wait_bounded(pvdone, (nt - 1) & 1, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, got)) {
+                if (lane == 0) fail();
+            } else {
+                tc_fence_after();
+                const int r = r0 + row;
+                const int j = h * geo.g + (live ? r / geo.C : 0), c = live ? r % geo.C : 0;
+                float *dst = fa.out + ((int64_t(b) * geo.Hq + j) * geo.C + c) * D;
+                const float il = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    float o[32];
+                    tmem_ld32(lane_base + 128u + uint32_t(cb * 32), o);
+                    if (live) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4 *>(dst + cb * 32 + i) =
+                                make_float4(o[i] * il, o[i + 1] * il, o[i + 2] * il, o[i + 3] * il);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 map: `rows` rows of `cols` elements, boxes of box_rows x 64.
+bool map2d(CUtensorMap *mp, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    auto enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(mp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct PrepPlan {
+    int Rp, Wp;
+    size_t q_bytes, k_bytes, v_bytes;
+};
+PrepPlan prep_plan(const Geom &geo)
+{
+    PrepPlan p;
+    const int64_t R = int64_t(geo.g) * geo.C;
+    p.Rp = int((R + kQRows - 1) / kQRows * kQRows);
+    p.Wp = int((geo.Wmax + kKeyTile - 1) / kKeyTile * kKeyTile);
+    const size_t BH = size_t(geo.B) * geo.Hkv;
+    p.q_bytes = (BH * p.Rp * geo.d * 2 + 255) / 256 * 256;
+    p.k_bytes = (BH * p.Wp * geo.d * 2 + 255) / 256 * 256;
+    p.v_bytes = p.k_bytes;
+    return p;
+}
+
+}  // namespace
+
+bool prefill_attn_tc_eligible(const Geom &geo)
+{
+    const int64_t R = int64_t(geo.g) * geo.C;
+    const int64_t BH = int64_t(geo.B) * geo.Hkv;
+    const PrepPlan p = prep_plan(geo);
+    return geo.dtype == REATT_BF16 && R > 8 && (geo.d == 64 || geo.d == 128) &&
+           BH * p.Wp < (int64_t(1) << 31) && BH * p.Rp < (int64_t(1) << 31) &&
+           BH * geo.d < (int64_t(1) << 31);
+}
+
+size_t prefill_attn_tc_ws_bytes(const Geom &geo)
+{
+    if (!prefill_attn_tc_eligible(geo)) return 0;
+    const PrepPlan p = prep_plan(geo);
+    return 2 * p.q_bytes + 2 * p.k_bytes + p.v_bytes;
+}
+
+cudaError_t launch_attend_prefill_tc(const Geom &geo, const void *q, const void *kc,
+                                     const void *vc, const void *kcur, const void *vcur,
+                                     const int32_t *sel, const float2 *tab, float *out,
+                                     void *scratch, void *ws, cudaStream_t st)
+{
+    const PrepPlan pp = prep_plan(geo);
+    uint8_t *base = static_cast<uint8_t *>(scratch);
+    PrepOut po;
+    po.qh = reinterpret_cast<__nv_bfloat16 *>(base);
+    po.ql = reinterpret_cast<__nv_bfloat16 *>(base + pp.q_bytes);
+    po.kh = reinterpret_cast<__nv_bfloat16 *>(base + 2 * pp.q_bytes);
+    po.kl = reinterpret_cast<__nv_bfloat16 *>(base + 2 * pp.q_bytes + pp.k_bytes);
+    po.vt = reinterpret_cast<__nv_bfloat16 *>(base + 2 * pp.q_bytes + 2 * pp.k_bytes);
+    po.Rp = pp.Rp;
+    po.Wp = pp.Wp;
+    const unsigned BH = unsigned(geo.B * geo.Hkv);
+    dim3 pgrid(unsigned(pp.Wp / kPrepRows + pp.Rp / kPrepRows), BH);
+    const uint16_t *q16 = static_cast<const uint16_t *>(q);
+    const uint16_t *k16 = static_cast<const uint16_t *>(kc), *v16 = static_cast<const uint16_t *>(vc);
+    const uint16_t *kq = static_cast<const uint16_t *>(kcur), *vq = static_cast<const uint16_t *>(vcur);
+    cudaError_t e;
+    if (geo.d == 128)
+        e = launch_pdl(prefill_prep_kernel<128>, pgrid, dim3(256), 0, st, geo, q16, k16, v16, kq, vq,
+                       sel, tab, po);
+    else
+        e = launch_pdl(prefill_prep_kernel<64>, pgrid, dim3(256), 0, st, geo, q16, k16, v16, kq, vq,
+                       sel, tab, po);
+    if (e != cudaSuccess) return e;
+    const uint64_t BHu = BH;
+    CUtensorMap qh, ql, kh, kl, vt;
+    if (!map2d(&qh, po.qh, BHu * pp.Rp, geo.d, kQRows) || !map2d(&ql, po.ql, BHu * pp.Rp, geo.d, kQRows) ||
+        !map2d(&kh, po.kh, BHu * pp.Wp, geo.d, kKeyTile) || !map2d(&kl, po.kl, BHu * pp.Wp, geo.d, kKeyTile) ||
+        !map2d(&vt, po.vt, BHu * geo.d, pp.Wp, uint32_t(geo.d)))
+        return cudaErrorInvalidValue;
+    FaArgs fa;
+    fa.out = out;
+    fa.sel = sel;
+    fa.Rp = pp.Rp;
+    fa.Wp = pp.Wp;
+    dim3 grid(unsigned(pp.Rp / kQRows), BH);
+    if (geo.d == 128) {
+        auto kern = attend_prefill_tc_kernel<128>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(FaSmem<128>::kBytes));
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(kern, grid, dim3(kFaThreads), FaSmem<128>::kBytes, st, qh, ql, kh, kl, vt, geo, fa, ws);
+    } else {
+        auto kern = attend_prefill_tc_kernel<64>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(FaSmem<64>::kBytes));
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(kern, grid, dim3(kFaThreads), FaSmem<64>::kBytes, st, qh, ql, kh, kl, vt, geo, fa, ws);
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace reatt

@@ -46,6 +46,14 @@ size_t prefill_tc_ws_bytes(const Geom &geo);
 cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, float *scores,
                               void *ws, void *scratch, cudaStream_t st);
 
+// prefill attention on tcgen05 (bf16, more than 8 query rows per KV head)
+bool prefill_attn_tc_eligible(const Geom &geo);
+size_t prefill_attn_tc_ws_bytes(const Geom &geo);
+cudaError_t launch_attend_prefill_tc(const Geom &geo, const void *q, const void *kc,
+                                     const void *vc, const void *kcur, const void *vcur,
+                                     const int32_t *sel, const float2 *tab, float *out,
+                                     void *scratch, void *ws, cudaStream_t st);
+
 // top-k: scratch holds per-slice candidates when NS is large; zero_words
 // (nullable) are cleared by the first CTA (used to reset attention tickets);
 // rope_tab (nullable) is filled by spare CTAs of the same launch

@@ -27,106 +27,19 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace reatt {
 
 namespace {
+
+using namespace tc;
 
 constexpr int kTcThreads = 6 * 32;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kTileM = 128;          // tokens per tile = TMEM lanes
 constexpr int kTileN = 128;          // queries per MMA tile = TMEM columns
 constexpr int kQStages = 4;          // query-tile ring
 constexpr uint32_t kTmemCols = 256;  // two accumulators
-constexpr int kBoxBytes = 128 * 128; // one 128-row x 64-element bf16 box (128 B rows)
-
-// ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols)
-{
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_addr(slot)),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish()
-{
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
-{
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before()
-{
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after()
-{
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-// D[tmem] (+)= A[smem desc] x B[smem desc]^T, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// The mbarrier gets one arrival when every tcgen05 op issued so far by this
-// thread has completed.
-__device__ __forceinline__ void tc_commit(uint64_t *bar)
-{
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_addr(bar))
-        : "memory");
-}
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-          "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-// 2-D tiled TMA load (no multicast); x is the innermost (element) coordinate.
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
-                                            uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
-        : "memory");
-}
-// Shared-memory matrix descriptor: K-major operand in 128-byte-swizzled 8-row
-// atoms (rows of 128 B, 8-row groups 1024 B apart), descriptor version 1.
-__device__ __forceinline__ uint64_t sw128_desc(const void *p)
-{
-    const uint64_t addr = smem_addr(p);
-    uint64_t d = (addr >> 4) & 0x3FFFull;    // start address
-    d |= 1ull << 16;                          // leading byte offset (unused: swizzled K-major)
-    d |= uint64_t(1024 >> 4) << 32;           // stride byte offset between 8-row groups
-    d |= 1ull << 46;                          // version
-    d |= 2ull << 61;                          // 128-byte swizzle
-    return d;
-}
-// Instruction descriptor, kind::f16: fp32 D, bf16 A and B, both K-major, M x N.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kTileN >> 3) << 17) |
-                            (uint32_t(kTileM >> 4) << 24);
 
 struct TcArgs {
     int64_t items;   // BH * ntiles
@@ -264,7 +177,7 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                             const uint64_t adesc = sw128_desc(ksm + bx * kBoxBytes) + uint64_t(kin * 2);
                             const uint64_t bdesc =
                                 sw128_desc(qsm + st * kQBytes + bx * kBoxBytes) + uint64_t(kin * 2);
-                            tc_mma(d_tmem, adesc, bdesc, kIdesc, (term | ks) != 0 ? 1u : 0u);
+                            tc_mma(d_tmem, adesc, bdesc, idesc_bf16(kTileM, kTileN), (term | ks) != 0 ? 1u : 0u);
                         }
                         tc_commit(&qempty[st]);   // stage free once these MMAs are done
                     }
