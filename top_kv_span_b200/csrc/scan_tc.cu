@@ -12,10 +12,11 @@
 // ~2^-17 relative -- one bf16 rounding of the sum would not be.  With g <= 2
 // query heads per KV head the raw bf16 heads are the terms instead (exact).
 //
-// Kernel: one CTA per SM, persistent over (head, 128-token tile) items.
+// Kernel: one CTA per SM, persistent over (head, 256-token) items: two K tiles
+// of 128 tokens share every query stage, halving the L2 bytes per MMA.
 //   warp 0  : TMA producer (cp.async.bulk.tensor, 128B swizzle, no multicast)
 //   warp 1  : TMEM allocation; one thread issues tcgen05.mma (M=128 tokens,
-//             N=128 queries, K=16) into two TMEM accumulators in turn
+//             N=128 queries, K=16) per K tile into two accumulator sets in turn
 //   warps 2-5: epilogue -- tcgen05.ld of the accumulator rows (one token row
 //             per thread), max over valid queries, then a segmented warp max
 //             over the span's tokens; only span scores reach global memory.
@@ -37,13 +38,14 @@ using namespace tc;
 
 constexpr int kTcThreads = 6 * 32;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int kTileM = 128;          // tokens per tile = TMEM lanes
+constexpr int kTiles = 2;            // token tiles per item: each query stage feeds both
 constexpr int kTileN = 128;          // queries per MMA tile = TMEM columns
 constexpr int kQStages = 4;          // query-tile ring
-constexpr uint32_t kTmemCols = 256;  // two accumulators
+constexpr uint32_t kTmemCols = 512;  // two accumulator sets of kTiles x 128 columns
 
 struct TcArgs {
     int64_t items;   // BH * ntiles
-    int ntiles;      // 128-token tiles per head
+    int ntiles;      // items (kTiles x 128 tokens) per head
     int nqt;         // 128-query tiles
     int nterms;      // bf16 terms per query
     int cpad;        // nqt * 128
@@ -57,7 +59,7 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 {
     constexpr int KS = D / 16;             // MMA k-steps over the head width
     constexpr int NBOX = D / 64;           // 64-element swizzle boxes per row
-    constexpr uint32_t kKBytes = NBOX * kBoxBytes;
+    constexpr uint32_t kKBytes = kTiles * NBOX * kBoxBytes;
     constexpr uint32_t kQBytes = NBOX * kBoxBytes;
     extern __shared__ uint8_t smem_raw[];
     // 128B-swizzled operand tiles want 1024-byte alignment
@@ -111,14 +113,17 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             for (int64_t it = blockIdx.x; ok && it < ta.items; it += gridDim.x) {
                 const int64_t bh = it / ta.ntiles;
                 const int tile = int(it % ta.ntiles);
-                const int y = int(bh * geo.T + geo.G + int64_t(tile) * kTileM);
+                const int y = int(bh * geo.T + geo.G + int64_t(tile) * kTiles * kTileM);
                 if (kuse > 0 && (aborted() || !mbar_wait_bounded(kempty, (kuse - 1) & 1, kWaitLimitNs))) {
                     fail();
                     ok = false;
                     break;
                 }
                 mbar_arrive_expect_tx(kfull, kKBytes);
-                for (int bx = 0; bx < NBOX; ++bx) tma_load_2d(ksm + bx * kBoxBytes, &kmap, 64 * bx, y, kfull);
+                for (int t = 0; t < kTiles; ++t)
+                    for (int bx = 0; bx < NBOX; ++bx)
+                        tma_load_2d(ksm + (t * NBOX + bx) * kBoxBytes, &kmap, 64 * bx,
+                                    y + t * kTileM, kfull);
                 ++kuse;
                 for (int qt = 0; ok && qt < ta.nqt; ++qt)
                     for (int term = 0; term < ta.nterms; ++term, ++qn) {
@@ -162,7 +167,7 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + uint32_t(acc * kTileN);
+                    const uint32_t d_tmem = tmem_base + uint32_t(acc * kTiles * kTileN);
                     for (int term = 0; term < ta.nterms; ++term, ++qn) {
                         const int st = int(qn % kQStages);
                         if (aborted() || !mbar_wait_bounded(&qfull[st], (qn / kQStages) & 1, kWaitLimitNs)) {
@@ -172,13 +177,17 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                         }
                         tc_fence_after();
 #pragma unroll
-                        for (int ks = 0; ks < KS; ++ks) {
-                            const int bx = ks / 4, kin = ks % 4;   // box, 32-byte step inside it
-                            const uint64_t adesc = sw128_desc(ksm + bx * kBoxBytes) + uint64_t(kin * 2);
-                            const uint64_t bdesc =
-                                sw128_desc(qsm + st * kQBytes + bx * kBoxBytes) + uint64_t(kin * 2);
-                            tc_mma(d_tmem, adesc, bdesc, idesc_bf16(kTileM, kTileN), (term | ks) != 0 ? 1u : 0u);
-                        }
+                        for (int t = 0; t < kTiles; ++t)
+#pragma unroll
+                            for (int ks = 0; ks < KS; ++ks) {
+                                const int bx = ks / 4, kin = ks % 4;   // box, 32-byte step inside it
+                                const uint64_t adesc =
+                                    sw128_desc(ksm + (t * NBOX + bx) * kBoxBytes) + uint64_t(kin * 2);
+                                const uint64_t bdesc =
+                                    sw128_desc(qsm + st * kQBytes + bx * kBoxBytes) + uint64_t(kin * 2);
+                                tc_mma(d_tmem + uint32_t(t * kTileN), adesc, bdesc,
+                                       idesc_bf16(kTileM, kTileN), (term | ks) != 0 ? 1u : 0u);
+                            }
                         tc_commit(&qempty[st]);   // stage free once these MMAs are done
                     }
                     if (ok) tc_commit(&accfull[acc]);
@@ -197,7 +206,9 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         for (int64_t it = blockIdx.x; it < ta.items; it += gridDim.x) {
             const int64_t bh = it / ta.ntiles;
             const int tile = int(it % ta.ntiles);
-            float tokmax = -INFINITY;
+            float tokmax[kTiles];
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) tokmax[t] = -INFINITY;
             bool ok = true;
             for (int qt = 0; qt < ta.nqt; ++qt, ++an) {
                 const int acc = int(an & 1);
@@ -209,15 +220,19 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     break;
                 }
                 tc_fence_after();
-                const uint32_t taddr = tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * kTileN);
 #pragma unroll
-                for (int ch = 0; ch < kTileN / 32; ++ch) {
-                    float v[32];
-                    tmem_ld32(taddr + uint32_t(ch * 32), v);
-                    const int c0 = qt * kTileN + ch * 32;
+                for (int t = 0; t < kTiles; ++t) {
+                    const uint32_t taddr = tmem_base + (uint32_t(quad * 32) << 16) +
+                                           uint32_t((acc * kTiles + t) * kTileN);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c0 + j < geo.C) tokmax = fmaxf(tokmax, v[j]);
+                    for (int ch = 0; ch < kTileN / 32; ++ch) {
+                        float v[32];
+                        tmem_ld32(taddr + uint32_t(ch * 32), v);
+                        const int c0 = qt * kTileN + ch * 32;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (c0 + j < geo.C) tokmax[t] = fmaxf(tokmax[t], v[j]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -225,10 +240,13 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             }
             if (!ok) break;
             // span max: S divides 32, tiles start on span boundaries
-            const int64_t moff = int64_t(tile) * kTileM + row;
-            float val = moff < geo.M ? tokmax : -INFINITY;
-            for (int o = 1; o < geo.S; o <<= 1) val = fmaxf(val, __shfl_xor_sync(0xffffffffu, val, o));
-            if (moff < geo.M && (lane % geo.S) == 0) scores[bh * geo.NS + moff / geo.S] = val;
+#pragma unroll
+            for (int t = 0; t < kTiles; ++t) {
+                const int64_t moff = (int64_t(tile) * kTiles + t) * kTileM + row;
+                float val = moff < geo.M ? tokmax[t] : -INFINITY;
+                for (int o = 1; o < geo.S; o <<= 1) val = fmaxf(val, __shfl_xor_sync(0xffffffffu, val, o));
+                if (moff < geo.M && (lane % geo.S) == 0) scores[bh * geo.NS + moff / geo.S] = val;
+            }
         }
     }
     tc_fence_before();
@@ -318,7 +336,7 @@ cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, fl
                               void *ws, void *scratch, cudaStream_t st)
 {
     TcArgs ta;
-    ta.ntiles = int((geo.M + kTileM - 1) / kTileM);
+    ta.ntiles = int((geo.M + kTiles * kTileM - 1) / (kTiles * kTileM));
     ta.items = int64_t(geo.B) * geo.Hkv * ta.ntiles;
     ta.nqt = (geo.C + kTileN - 1) / kTileN;
     ta.cpad = ta.nqt * kTileN;
@@ -342,7 +360,7 @@ cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, fl
     int grid = num_sms();
     if (ta.items < grid) grid = int(ta.items);
     const size_t box = kBoxBytes;
-    const size_t smem = 1024 + (geo.d / 64) * box * (1 + kQStages) + (2 + 2 * kQStages + 5) * 8 + 16;
+    const size_t smem = 1024 + (geo.d / 64) * box * (kTiles + kQStages) + (2 + 2 * kQStages + 5) * 8 + 16;
     if (geo.d == 128) {
         auto kern = scan_prefill_tc_kernel<128>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
