@@ -172,6 +172,16 @@ REATT_API int reatt_step(const reatt_dims *dims, const void *q, const void *k_ca
                reatt_stream stream);
 
 /*
+ * Diagnostic for the failure-detection path: launches one thread that waits
+ * on an mbarrier nothing completes, bounded by limit_ns (0 < limit_ns <= 10 s),
+ * after which it records REATT_ETIMEOUT in the workspace status word and
+ * returns.  No fault, trap or hang; the context stays usable.  Read the
+ * result with reatt_workspace_status().  EINVAL for a null/misaligned ws or
+ * a limit out of range.
+ */
+REATT_API int reatt_selftest_bounded_wait(void *ws, int64_t limit_ns, reatt_stream stream);
+
+/*
  * reatt_step without a caller-supplied workspace.  The pages have no
  * counterpart to this call; it exists for callers that cannot allocate device
  * memory: a plugin interface that gives its kernels no allocator, or a

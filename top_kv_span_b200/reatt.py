@@ -20,7 +20,7 @@ F32, BF16 = 0, 1
 
 EXPORTS = ["reatt_status_string", "reatt_num_spans", "reatt_window_max", "reatt_workspace_bytes",
            "reatt_workspace_status", "reatt_score_spans", "reatt_topk", "reatt_gather_rope",
-           "reatt_attend", "reatt_step", "reatt_step_fixed_scratch"]
+           "reatt_attend", "reatt_step", "reatt_selftest_bounded_wait", "reatt_step_fixed_scratch"]
 
 
 class reatt_dims(ctypes.Structure):
@@ -54,6 +54,7 @@ lib.reatt_gather_rope.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _
 lib.reatt_attend.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.reatt_step.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.reatt_step_fixed_scratch.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.reatt_selftest_bounded_wait.argtypes = [_vp, ctypes.c_int64, _vp]
 for _name in EXPORTS[1:]:
     getattr(lib, _name).restype = ctypes.c_int
 
@@ -166,6 +167,15 @@ def reatt_step(dims, q, k_cache, v_cache, k_cur, v_cur, sel_out, out, ws, stream
                         _ptr(v_cur), _ptr(sel_out), _ptr(out), _ptr(ws), _stream(stream))
     if check:
         _check(rc, "reatt_step")
+    return rc
+
+
+def reatt_selftest_bounded_wait(ws, limit_ns, stream=None, check=True):
+    """Run one bounded wait that nothing completes; the timeout lands in the
+    workspace status word (read it with reatt_workspace_status)."""
+    rc = lib.reatt_selftest_bounded_wait(_ptr(ws), int(limit_ns), _stream(stream))
+    if check:
+        _check(rc, "reatt_selftest_bounded_wait")
     return rc
 
 
