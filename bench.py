@@ -29,7 +29,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ReAttention step latency (µs) and KV-scan GB/s vs HBM peak at 128K–4M context"
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "scan_decode_llama3_8b_128k.md")
+# committed ncu summaries holding the dominant kernel's per-launch DRAM traffic
+PROFILE_SUMMARY = {
+    "llama3_8b_128k": os.path.join(ROOT, "profiles", "scan_decode_llama3_8b_128k.md"),
+    "llama3_8b_prefill_256k": os.path.join(ROOT, "profiles",
+                                           "scan_prefill_tc_llama3_8b_prefill_256k.md"),
+}
 
 
 def step_bytes(w):
@@ -44,12 +49,15 @@ def step_bytes(w):
     return scan, scan + window + io
 
 
-def read_traffic():
+def read_traffic(workload):
     """Per-launch DRAM traffic of the scan kernel from the committed ncu
-    summary (a line 'traffic_bytes_per_launch: N', with the kernel build it was
-    taken on); None if absent."""
+    summary of this workload (a line 'traffic_bytes_per_launch: N', with the
+    kernel build it was taken on); None if there is none."""
+    path = PROFILE_SUMMARY.get(workload)
+    if path is None:
+        return None
     try:
-        with open(PROFILE_SUMMARY) as f:
+        with open(path) as f:
             for line in f:
                 if line.startswith("traffic_bytes_per_launch:"):
                     v = line.split(":", 1)[1].strip()
@@ -136,12 +144,40 @@ def aggregate(world, step_b, steps, total_ms, e2e_ms, scan_ms, reduce_max=None):
 
 
 def peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, kind): the measured copy bandwidth and
+    cuBLAS bf16 throughput of this machine's B200s, else the earlier fallback."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
     except Exception:
-        return 6650.0, "fallback"
+        return 6650.0, 1590.0, "fallback"
+
+
+def scan_flops(w):
+    """Algorithmic flops of the prefill scan in the summed-query form: one
+    length-d dot product per (query position, middle token, KV head)."""
+    M = max(0, w.T - w.G - w.L)
+    return 2 * w.B * w.Hkv * w.C * M * w.d
+
+
+def roofline(w, scan_b, scan_ms):
+    """Roofline entry of the dominant kernel (the span scan): HBM-bound in
+    decode, tensor-bound (tcgen05) for a bf16 prefill chunk."""
+    hbm, tflops, kind = peaks()
+    traffic = read_traffic(w.name)
+    if w.C > 1 and w.dtype == "bf16" and 32 % w.S == 0:
+        achieved = scan_flops(w) / (scan_ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": round(achieved, 1), "peak": tflops,
+                "peak_kind": kind + " (bf16 burst)", "unit": "TFLOP/s",
+                "frac": round(achieved / tflops, 4), "traffic": traffic,
+                "kernel": "scan_prefill_tc_kernel", "flops_per_launch": scan_flops(w),
+                "note": "issued MMA work is 2x (bf16 hi + lo query terms)"}
+    achieved = scan_b / (scan_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "peak_kind": kind,
+            "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic,
+            "kernel": "scan_decode_kernel" if w.C == 1 else "scan_multi_kernel",
+            "bytes_per_launch": scan_b}
 
 
 def dist_setup(n_gpus):
@@ -273,7 +309,6 @@ def run_ours(args):
     total_ms, e2e_ms, scan_ms = agg["total_ms"], agg["e2e_ms"], agg["scan_ms"]
     ms_per_step = total_ms / args.steps
     value, e2e_value = agg["value"], agg["e2e_value"]
-    peak, peak_kind = peaks()
     achieved = scan_b / (scan_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC,
@@ -295,10 +330,7 @@ def run_ours(args):
                    "T": w.T, "G": w.G, "L": w.L, "S": w.S, "k": w.k, "rope_base": w.rope_base,
                    "parallelism": f"replicas x{world}",
                    "l2": "flushed before every step (512 MiB read); flush outside the step events"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": read_traffic(), "kernel": "scan_decode_kernel",
-                     "bytes_per_launch": scan_b},
+        "roofline": roofline(w, scan_b, scan_ms),
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms / args.steps * 1e3, 2)},
         "gpu_launches": per_step * args.steps,

@@ -28,6 +28,10 @@ CASES = {
     # ragged: M = 983 = 140*7 + 3, two sequences, GQA 3
     "odd_f32_d64": TINY.replace(name="odd", B=2, Hq=6, Hkv=2, T=1003, G=3, L=17, S=7, k=5,
                                 n_needles=2, seed=11),
+    # middle a whole number of spans (M = 987 = 141*7): the window length is
+    # known before the selection, so the decode attention starts early
+    "early_f32_gqa3": TINY.replace(name="early", B=2, Hq=6, Hkv=2, T=1007, G=3, L=17, S=7, k=5,
+                                   n_needles=2, seed=27),
     "bf16_d128_20k": LLAMA.replace(name="bf16_20k", Hq=8, Hkv=2, T=20000, L=512, k=16,
                                    n_needles=3, seed=12),
     "bf16_d64_ragged": LLAMA.replace(name="bf16_d64", Hq=4, Hkv=2, d=64, T=9001, G=5, L=300,

@@ -173,7 +173,8 @@ int reatt_score_spans(const reatt_dims *dims, const void *q, const void *k_cache
         return REATT_EINVAL;
     const WsPlan p = ws_plan(g);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return cuda_status(launch_score_spans(g, q, k_cache, span_scores, ws, at(ws, p.qsum), st));
+    return cuda_status(
+        launch_score_spans(g, q, k_cache, span_scores, ws, at(ws, p.qsum), nullptr, st));
 }
 
 int reatt_topk(const reatt_dims *dims, const float *span_scores, int32_t *sel, void *ws,
@@ -245,18 +246,27 @@ int reatt_step(const reatt_dims *dims, const void *q, const void *k_cache, const
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float *scores = reinterpret_cast<float *>(at(ws, p.scores));
     int32_t *sel = sel_out ? sel_out : reinterpret_cast<int32_t *>(at(ws, p.sel));
-    cudaError_t e = launch_score_spans(g, q, k_cache, scores, ws, at(ws, p.qsum), st);
-    if (e != cudaSuccess) return REATT_ECUDA;
-    // the top-k launch also clears the attention tickets and fills the RoPE table
     float2 *tab = reinterpret_cast<float2 *>(at(ws, p.tab));
-    e = launch_topk(g, scores, sel, at(ws, p.topk), reinterpret_cast<uint32_t *>(at(ws, p.ticket)),
-                    int(p.ticket_bytes / sizeof(uint32_t)), tab, st);
+    // Decode with a window length that does not depend on the selection: the
+    // scan writes the RoPE table and the attention starts on the fixed part
+    // of the window while the top-k runs.  Otherwise the top-k launch fills
+    // the table.  Either way the top-k launch clears the attention tickets.
+    const bool tc_attn = prefill_attn_tc_eligible(g);
+    const int64_t w_known = (g.C == 1 && g.NS > 0 && !tc_attn && attn_plan(g).decode)
+                                ? decode_window_known(g)
+                                : -1;
+    cudaError_t e = launch_score_spans(g, q, k_cache, scores, ws, at(ws, p.qsum),
+                                       w_known >= 0 ? tab : nullptr, st);
     if (e != cudaSuccess) return REATT_ECUDA;
-    if (prefill_attn_tc_eligible(g))   // many query rows: tensor-core attention
+    e = launch_topk(g, scores, sel, at(ws, p.topk), reinterpret_cast<uint32_t *>(at(ws, p.ticket)),
+                    int(p.ticket_bytes / sizeof(uint32_t)), w_known >= 0 ? nullptr : tab, st);
+    if (e != cudaSuccess) return REATT_ECUDA;
+    if (tc_attn)   // many query rows: tensor-core attention
         return cuda_status(launch_attend_prefill_tc(g, q, k_cache, v_cache, k_cur, v_cur, sel, tab,
                                                     out, at(ws, p.fa), ws, st));
     return cuda_status(launch_attend(g, q, nullptr, nullptr, nullptr, k_cache, v_cache, k_cur,
-                                     v_cur, sel, tab, out, at(ws, p.ticket), ws, true, st));
+                                     v_cur, sel, tab, out, at(ws, p.ticket), ws, true, st,
+                                     w_known));
 }
 
 }  // extern "C"

@@ -33,7 +33,6 @@ namespace {
 constexpr int kAttnThreads = 256;
 constexpr int kKT = 64;                 // keys per tile
 constexpr int kTargetCtas = 296;        // tile kernel: ~2 CTAs per SM (148 SMs)
-constexpr int kDecodeCtas = 148;        // decode kernels: ~1 CTA per SM
 constexpr int kMinSplitKeys = 128;      // keys per split at least
 
 struct WinMap {
@@ -147,6 +146,7 @@ struct AttnArgs {
     float2 *part_ml;          // [BH][nqb][nsplit][QB] (max, sum)
     uint32_t *ticket;         // [BH][nqb]
     int nqb, nsplit;
+    int64_t w_known;          // staged decode: window length known before the selection, or -1
 };
 
 __device__ __forceinline__ WinMap attn_winmap(const Geom &geo, const AttnArgs &a, bool virt,
@@ -651,32 +651,71 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
         mbar_init_fence();
     }
     if (tid < D / 2) freq[tid] = make_float2(geo.rope_hi[tid], geo.rope_lo[tid]);
-    pdl_wait();   // the selection (and tickets) come from the preceding kernels
+    // With the window length known up front, the rows that do not depend on
+    // the selection (local part and current token) are taken first, while the
+    // top-k still runs; only the producer's copies of chosen rows and the
+    // split merge wait for the preceding grid.  Otherwise everything waits.
+    const bool early = a.w_known >= 0;
+    if (!early) pdl_wait();
 
     const int split = blockIdx.x;
     const int64_t bh = blockIdx.z;
     const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv);
     const int nrows = geo.g * geo.C;
     const int32_t *sel_bh = a.sel + bh * geo.k;
-    const WinMap m = make_winmap(geo, sel_bh);
+    WinMap m;
+    if (early) {
+        m.g_end = geo.g_end;
+        m.loc_begin = geo.loc_begin;
+        m.n_loc = geo.n_loc;
+        m.W = a.w_known;
+        m.nsel_rows = m.W - m.g_end - m.n_loc - geo.C;
+    } else {
+        m = make_winmap(geo, sel_bh);
+    }
     const int64_t W = m.W, qpos0 = W - geo.C;
-    int64_t kbeg64, kend64;
-    split_range(geo, W, a.nsplit, split, 0, nrows, CH, kbeg64, kend64);
-    const int kbeg = int(kbeg64), kend = int(kend64);
-    // span ids of the chosen part inside [kbeg, kend)
     const int g_end = int(m.g_end), nsel = int(m.nsel_rows), nloc = int(m.n_loc);
+    // This CTA's rows: a slice of the early range [g_end + nsel, W), then a
+    // slice of the late range [0, g_end + nsel) (without early mode the late
+    // range is the whole window), cut at multiples of CH; rows past the last
+    // query's causal limit are dropped.
+    const int r_mid = early ? g_end + nsel : int(W);
+    int eb, ee, lb, le;
+    {
+        const int last_row = nrows - 1;
+        const int c_max = (last_row / geo.C == 0) ? last_row % geo.C : geo.C - 1;
+        const int lim = int(W) - geo.C + c_max + 1;
+        auto part = [&](int r0, int r1, int &pb, int &pe) {
+            int len = (r1 - r0 + a.nsplit - 1) / a.nsplit;
+            len = (len + CH - 1) / CH * CH;
+            pb = r0 + split * len;
+            pe = pb + len;
+            if (pe > r1) pe = r1;
+            if (pe > lim) pe = lim;
+            if (pb > pe) pb = pe;
+        };
+        part(r_mid, int(W), eb, ee);
+        part(0, r_mid, lb, le);
+    }
+    const int nE = (ee - eb + CH - 1) / CH;
+    const int nchunks = nE + (le - lb + CH - 1) / CH;
+    // chunk ci -> first window row and row count
+    auto chunk_at = [&](int ci, int &p0, int &n) {
+        const int pend = ci < nE ? ee : le;
+        p0 = ci < nE ? eb + ci * CH : lb + (ci - nE) * CH;
+        n = pend - p0 < CH ? pend - p0 : CH;
+    };
+    // span ids of the chosen part inside the late slice
     int j0 = 0, jn = 0;
     {
-        const int lo = kbeg > g_end ? kbeg : g_end;
-        const int hi = kend < g_end + nsel ? kend : g_end + nsel;
+        const int lo = lb > g_end ? lb : g_end;
+        const int hi = le < g_end + nsel ? le : g_end + nsel;
         if (lo < hi) {
             j0 = (lo - g_end) / geo.S;
             jn = (hi - 1 - g_end) / geo.S - j0 + 1;
         }
     }
     const bool sel_cached = jn <= kSelCache;
-    if (sel_cached)
-        for (int j = tid; j < jn; j += blockDim.x) sel_s[j] = sel_bh[j0 + j];
     __syncthreads();   // freq visible to the query rotation
     for (int x = tid; x < RP * (D / 2); x += blockDim.x) {
         const int rr = x / (D / 2), i = x % (D / 2);
@@ -687,27 +726,29 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
     }
     __syncthreads();
 
-    const int nchunks = kend > kbeg ? (kend - kbeg + CH - 1) / CH : 0;
     if (warp == kTmaCW) {
         // ------------------------------------------------ producer warp
-        // chunk ci = window rows [kbeg + ci*CH, +CH) -> stage ci % kTmaStages;
-        // lane l issues every chunk of stage l, in order, so each barrier has
-        // one waiter taking its phases in turn.  A chunk crossing a region
-        // boundary is copied as several runs.
+        // chunk ci -> stage ci % kTmaStages; lane l issues every chunk of
+        // stage l, in order, so each barrier has one waiter taking its phases
+        // in turn.  A chunk crossing a region boundary is copied as several
+        // runs.  Chunks of the early slice come first; before the first chunk
+        // of the late slice the warp waits for the selection.
         static_assert(kTmaStages <= 32, "one producer lane per stage");
-        if (lane < kTmaStages) {
-            int issued = 0;
-            for (int ci = lane; ci < nchunks; ci += kTmaStages, ++issued) {
+        int issued = 0, ci = lane;
+        bool stop = lane >= kTmaStages;
+        auto issue_until = [&](int c_end) {
+            for (; !stop && ci < c_end; ci += kTmaStages, ++issued) {
                 const int stage = lane;
                 if (issued > 0 &&
                     (*(volatile int *)&abort_flag ||
                      !mbar_wait_bounded(&empty[stage], uint32_t((issued - 1) & 1), kWaitLimitNs))) {
                     report_status(ws, REATT_ETIMEOUT);
                     *(volatile int *)&abort_flag = 1;
+                    stop = true;
                     break;
                 }
-                const int p0 = kbeg + ci * CH;
-                const int n = kend - p0 < CH ? kend - p0 : CH;
+                int p0, n;
+                chunk_at(ci, p0, n);
                 uint8_t *dst = ring + stage * Sh::kStageBytes;
                 mbar_arrive_expect_tx(&full[stage], uint32_t(n) * (2u * RB + Sh::kTabRowBytes));
                 bulk_load_plain(dst + 2 * CH * RB, a.tab + int64_t(p0) * (D / 2),
@@ -738,10 +779,18 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
                     p += r;
                 }
             }
-            // drain: this stage's last issued copy has landed
-            if (issued > 0 && !mbar_wait_bounded(&full[lane], uint32_t((issued - 1) & 1), kWaitLimitNs))
-                report_status(ws, REATT_ETIMEOUT);
-        }
+        };
+        issue_until(nE);
+        __syncwarp();
+        pdl_wait();   // the selection comes from the preceding kernel
+        if (sel_cached)
+            for (int j = lane; j < jn; j += 32) sel_s[j] = sel_bh[j0 + j];
+        __syncwarp();
+        issue_until(nchunks);
+        // drain: this stage's last issued copy has landed
+        if (lane < kTmaStages && issued > 0 &&
+            !mbar_wait_bounded(&full[lane], uint32_t((issued - 1) & 1), kWaitLimitNs))
+            report_status(ws, REATT_ETIMEOUT);
     } else {
         // ---------------------------------------------------- consumers
         float qlo[RP][PD], qhi[RP][PD];
@@ -768,8 +817,8 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
 
         for (int ci = warp; ci < nchunks; ci += kTmaCW) {
             const int stage = ci % kTmaStages;
-            const int p0 = kbeg + ci * CH;
-            const int n = kend - p0 < CH ? kend - p0 : CH;
+            int p0, n;
+            chunk_at(ci, p0, n);
             if (__any_sync(0xffffffffu, *(volatile int *)&abort_flag != 0)) break;
             const bool ok =
                 mbar_wait_bounded(&full[stage], uint32_t((ci / kTmaStages) & 1), kWaitLimitNs);
@@ -893,6 +942,7 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
             }
         }
     }
+    pdl_wait();   // split partials and tickets: after the preceding grid (it clears the tickets)
     __syncthreads();
     // merge the consumer warps
     if (tid < RP) {
@@ -1270,7 +1320,7 @@ cudaError_t launch_decode_attn(const Geom &geo, const AttnArgs &a, int RP, const
 
 }  // namespace
 
-AttnPlan attn_plan(const Geom &geo)
+AttnPlan attn_plan(const Geom &geo, int reserved_sms)
 {
     AttnPlan p;
     const int64_t R = int64_t(geo.g) * geo.C;
@@ -1279,8 +1329,9 @@ AttnPlan attn_plan(const Geom &geo)
         p.decode = true;
         p.QB = R <= 1 ? 1 : R <= 2 ? 2 : R <= 4 ? 4 : 8;
         p.nqb = 1;
-        // one wave: the staged kernel holds one CTA per SM
-        int64_t ns = kDecodeCtas / BH;
+        // one wave: the staged kernel holds one CTA per SM (on the SMs the
+        // kernels running beside it leave free)
+        int64_t ns = (num_sms() - reserved_sms) / BH;
         const int64_t max_split = (geo.Wmax + kMinSplitKeys - 1) / kMinSplitKeys;
         const int64_t cap = int64_t(kDecWarps - 1) * geo.d;   // combine scratch (floats / QB)
         if (ns > max_split) ns = max_split;
@@ -1347,9 +1398,16 @@ cudaError_t launch_attend(const Geom &geo, const void *q, const float *kw, const
                           const int32_t *win_len, const void *kc, const void *vc,
                           const void *kcur, const void *vcur, const int32_t *sel,
                           const float2 *rope_tab, float *out, void *scratch, void *ws, bool virt,
-                          cudaStream_t st)
+                          cudaStream_t st, int64_t w_known)
 {
-    const AttnPlan p = attn_plan(geo);
+    // Early mode: the selecting top-k CTAs run beside the attention, so the
+    // split count leaves their SMs free (when they are few).
+    int reserved = 0;
+    if (w_known >= 0) {
+        const int t = topk_selecting_ctas(geo);
+        if (t < num_sms() / 2) reserved = t;
+    }
+    const AttnPlan p = attn_plan(geo, reserved);
     size_t tb = 0, mo = 0;
     attend_ws_bytes(geo, &tb, &mo);
     AttnArgs a;
@@ -1363,6 +1421,7 @@ cudaError_t launch_attend(const Geom &geo, const void *q, const float *kw, const
     a.part_ml = reinterpret_cast<float2 *>(static_cast<uint8_t *>(scratch) + mo);
     a.nqb = p.nqb;
     a.nsplit = p.nsplit;
+    a.w_known = (p.decode && virt) ? w_known : -1;
 #define REATT_ATT(T, D)                                                                        \
     do {                                                                                       \
         if (p.decode) {                                                                        \
@@ -1387,6 +1446,13 @@ cudaError_t launch_attend(const Geom &geo, const void *q, const float *kw, const
     if (geo.d == 128) REATT_ATT(float, 128);
     REATT_ATT(float, 64);
 #undef REATT_ATT
+}
+
+int64_t decode_window_known(const Geom &geo)
+{
+    const int64_t keff = geo.k < geo.NS ? geo.k : geo.NS;
+    if (keff > 0 && geo.M % geo.S != 0) return -1;   // the ragged last span may be chosen
+    return geo.g_end + keff * geo.S + geo.n_loc + geo.C;
 }
 
 }  // namespace reatt

@@ -35,10 +35,11 @@ inline bool geo_is_bf16(const Geom &g) { return g.dtype == REATT_BF16; }
 
 int num_sms();
 
-// span scoring: scratch holds the fp32 summed queries when C > 1
+// span scoring: scratch holds the fp32 summed queries when C > 1; rope_tab
+// (nullable, decode only) is filled with the step's RoPE table on the side
 size_t score_spans_ws_bytes(const Geom &geo);
 cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, float *scores,
-                               void *ws, void *scratch, cudaStream_t st);
+                               void *ws, void *scratch, float2 *rope_tab, cudaStream_t st);
 
 // prefill span scoring on tcgen05 (bf16, C > 1, S divides 32)
 bool prefill_tc_eligible(const Geom &geo);
@@ -58,6 +59,7 @@ cudaError_t launch_attend_prefill_tc(const Geom &geo, const void *q, const void 
 // (nullable) are cleared by the first CTA (used to reset attention tickets);
 // rope_tab (nullable) is filled by spare CTAs of the same launch
 size_t topk_ws_bytes(const Geom &geo);
+int topk_selecting_ctas(const Geom &geo);   // CTAs of the first top-k launch that select
 cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void *scratch,
                         uint32_t *zero_words, int nzero, float2 *rope_tab, cudaStream_t st);
 
@@ -69,7 +71,8 @@ struct AttnPlan {
     bool decode;   // warp kernel (<= 8 query rows per KV head) or tile kernel
     int QB, nqb, nsplit;
 };
-AttnPlan attn_plan(const Geom &geo);
+// reserved_sms: SMs left to kernels that run beside the attention (the top-k)
+AttnPlan attn_plan(const Geom &geo, int reserved_sms = 0);
 // bytes of tickets (256-aligned, reported separately) + split-K partials
 // (accumulators, then (max, sum) pairs at *ml_off)
 size_t attend_ws_bytes(const Geom &geo, size_t *ticket_bytes, size_t *ml_off);
@@ -81,6 +84,12 @@ cudaError_t launch_attend(const Geom &geo, const void *q, const float *kw, const
                           const int32_t *win_len, const void *kc, const void *vc,
                           const void *kcur, const void *vcur, const int32_t *sel,
                           const float2 *rope_tab, float *out, void *scratch, void *ws, bool virt,
-                          cudaStream_t st);
+                          cudaStream_t st, int64_t w_known = -1);
+// Window length of the fused decode step when it does not depend on the
+// selection (no ragged last span, or nothing selected), else -1.  With it the
+// decode attention takes the fixed part of the window (local rows and the
+// current token) before the selection is complete; the RoPE table must then
+// be written by the scan.
+int64_t decode_window_known(const Geom &geo);
 
 }  // namespace reatt

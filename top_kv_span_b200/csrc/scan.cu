@@ -119,7 +119,8 @@ __device__ __forceinline__ bool next_item(const Geom &geo, int64_t &gs, int64_t 
 template <typename T, int D>
 __global__ void __launch_bounds__(kScanThreads, kCtasPerSm)
 scan_decode_kernel(Geom geo, const T *__restrict__ q, const T *__restrict__ kc,
-                   float *__restrict__ scores, void *ws, int64_t spans_per_cta)
+                   float *__restrict__ scores, void *ws, int64_t spans_per_cta,
+                   float2 *__restrict__ rope_tab)
 {
     using Sh = ScanShape<T, D>;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -200,6 +201,22 @@ scan_decode_kernel(Geom geo, const T *__restrict__ q, const T *__restrict__ kc,
     }
 
     // ---------------------------------------------------- consumers
+    if (rope_tab) {
+        // The step's RoPE cos/sin table (tab[p*(D/2) + i] for window positions
+        // p < Wmax), written while the first ring stages are in flight so the
+        // attention can use it without waiting for the selection.  The grid
+        // stride is a multiple of D/2, so each thread keeps one frequency.
+        constexpr int kHalf = D / 2;
+        static_assert(kConsumers % kHalf == 0, "one frequency per consumer thread");
+        const float fhi = geo.rope_hi[tid % kHalf], flo = geo.rope_lo[tid % kHalf];
+        const int64_t n = geo.Wmax * kHalf;
+        for (int64_t x = int64_t(blockIdx.x) * kConsumers + tid; x < n;
+             x += int64_t(gridDim.x) * kConsumers) {
+            float c, s;
+            rope_cs(x / kHalf, fhi, flo, c, s);
+            rope_tab[x] = make_float2(c, s);
+        }
+    }
     const int gq = lane / Sh::kLpt, p = lane % Sh::kLpt;
     int stage = 0;
     uint32_t phase = 0;
@@ -395,7 +412,7 @@ scan_multi_kernel(Geom geo, const float *__restrict__ qsum, const T *__restrict_
 
 template <typename T, int D>
 cudaError_t launch_decode(const Geom &geo, const void *q, const void *kc, float *scores, void *ws,
-                          cudaStream_t st)
+                          float2 *rope_tab, cudaStream_t st)
 {
     using Sh = ScanShape<T, D>;
     const int64_t total = int64_t(geo.B) * geo.Hkv * geo.NS;
@@ -408,7 +425,7 @@ cudaError_t launch_decode(const Geom &geo, const void *q, const void *kc, float 
                                          int(Sh::kSmem));
     if (e != cudaSuccess) return e;
     scan_decode_kernel<T, D><<<grid, kScanThreads, Sh::kSmem, st>>>(
-        geo, static_cast<const T *>(q), static_cast<const T *>(kc), scores, ws, per);
+        geo, static_cast<const T *>(q), static_cast<const T *>(kc), scores, ws, per, rope_tab);
     return cudaGetLastError();
 }
 
@@ -438,16 +455,18 @@ size_t score_spans_ws_bytes(const Geom &geo)
 }
 
 cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, float *scores,
-                               void *ws, void *scratch, cudaStream_t st)
+                               void *ws, void *scratch, float2 *rope_tab, cudaStream_t st)
 {
     if (int64_t(geo.B) * geo.Hkv * geo.NS == 0) return cudaSuccess;
     if (geo.C == 1) {
         if (geo.d == 128)
-            return geo_is_bf16(geo) ? launch_decode<uint16_t, 128>(geo, q, kc, scores, ws, st)
-                                    : launch_decode<float, 128>(geo, q, kc, scores, ws, st);
-        return geo_is_bf16(geo) ? launch_decode<uint16_t, 64>(geo, q, kc, scores, ws, st)
-                                : launch_decode<float, 64>(geo, q, kc, scores, ws, st);
+            return geo_is_bf16(geo)
+                       ? launch_decode<uint16_t, 128>(geo, q, kc, scores, ws, rope_tab, st)
+                       : launch_decode<float, 128>(geo, q, kc, scores, ws, rope_tab, st);
+        return geo_is_bf16(geo) ? launch_decode<uint16_t, 64>(geo, q, kc, scores, ws, rope_tab, st)
+                                : launch_decode<float, 64>(geo, q, kc, scores, ws, rope_tab, st);
     }
+    if (rope_tab) return cudaErrorInvalidValue;   // only the decode scan writes the table
     if (prefill_tc_eligible(geo))   // tensor-core contraction (tcgen05 / TMEM)
         return launch_prefill_tc(geo, q, kc, scores, ws, scratch, st);
     float *qsum = static_cast<float *>(scratch);

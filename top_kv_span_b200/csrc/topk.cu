@@ -415,6 +415,11 @@ TopkPlan topk_plan(const Geom &geo)
 
 }  // namespace
 
+int topk_selecting_ctas(const Geom &geo)
+{
+    return geo.k == 0 ? 0 : geo.B * geo.Hkv * topk_plan(geo).nslices;
+}
+
 size_t topk_ws_bytes(const Geom &geo)
 {
     const TopkPlan p = topk_plan(geo);
