@@ -34,6 +34,15 @@ CASES = {
                                    n_needles=2, seed=27),
     "bf16_d128_20k": LLAMA.replace(name="bf16_20k", Hq=8, Hkv=2, T=20000, L=512, k=16,
                                    n_needles=3, seed=12),
+    # decode on the tensor cores with a few current tokens (causal among them)
+    # and with one query head per KV head
+    "decode_tc_c3": LLAMA.replace(name="dtc_c3", Hq=4, Hkv=2, C=3, T=32 + 256 + 32 * 210,
+                                  L=256, k=10, n_needles=1, seed=28),
+    "decode_tc_g1": LLAMA.replace(name="dtc_g1", Hq=2, Hkv=2, T=8 + 200 + 16 * 550, G=8, L=200,
+                                  S=16, k=12, n_needles=2, seed=29),
+    # bf16, d = 128, ragged last span: the CUDA-core staged decode kernel
+    "bf16_d128_ragged_staged": LLAMA.replace(name="bf16_rg", Hq=8, Hkv=2, T=20003, L=512, k=16,
+                                             n_needles=2, seed=30),
     "bf16_d64_ragged": LLAMA.replace(name="bf16_d64", Hq=4, Hkv=2, d=64, T=9001, G=5, L=300,
                                      S=32, k=12, n_needles=2, seed=13),
     "k_ge_ns_full_attention": LLAMA.replace(name="kge", Hq=8, Hkv=2, T=300, G=16, L=128, k=8,

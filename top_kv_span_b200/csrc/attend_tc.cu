@@ -533,6 +533,12 @@ PrepPlan prep_plan(const Geom &geo)
 
 }  // namespace
 
+bool encode_bf16_map(CUtensorMap *mp, const void *base, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows)
+{
+    return map2d(mp, base, rows, cols, box_rows);
+}
+
 bool prefill_attn_tc_eligible(const Geom &geo)
 {
     const int64_t R = int64_t(geo.g) * geo.C;

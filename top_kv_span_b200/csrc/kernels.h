@@ -1,6 +1,7 @@
 // Host-side launchers of the sm_100a kernels (internal to the library).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -66,6 +67,33 @@ cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void
 cudaError_t launch_gather_rope(const Geom &geo, const void *kc, const void *vc, const void *kcur,
                                const void *vcur, const int32_t *sel, float *kw, float *vw,
                                int32_t *win_len, cudaStream_t st);
+
+// Arguments of the windowed-attention kernels.
+struct AttnArgs {
+    const void *q;
+    const int32_t *sel;       // virtual window
+    const int32_t *win_len;   // materialised window
+    const float2 *tab;        // virtual window: RoPE cos/sin [Wmax][D/2]
+    float *out;
+    float *part_acc;          // [BH][nqb][nsplit][QB][D]
+    float2 *part_ml;          // [BH][nqb][nsplit][QB] (max, sum)
+    uint32_t *ticket;         // [BH][nqb]
+    int nqb, nsplit;
+    int64_t w_known;          // decode: window length known before the selection, or -1
+};
+
+// 2-D tensor map of a row-major bf16 matrix (rows x cols), boxes of
+// box_rows x 64 elements, 128-byte swizzle, zero fill out of range.
+bool encode_bf16_map(CUtensorMap *mp, const void *base, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows);
+
+// Decode attention of the fused step on the tensor cores (bf16, d = 128, at
+// most 8 query rows per KV head, every window run a multiple of 8 rows):
+// QB = RP query rows per CTA.
+bool decode_tc_eligible(const Geom &geo);
+cudaError_t launch_attend_decode_tc(const Geom &geo, const AttnArgs &a, int RP, const void *kc,
+                                    const void *vc, const void *kcur, const void *vcur, void *ws,
+                                    cudaStream_t st);
 
 struct AttnPlan {
     bool decode;   // warp kernel (<= 8 query rows per KV head) or tile kernel

@@ -83,6 +83,11 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
         : "memory");
 }
+// Bring a tensor map (kernel parameter) into the descriptor cache ahead of use.
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 // Shared-memory matrix descriptor: K-major operand in 128-byte-swizzled 8-row
 // atoms (rows of 128 B, 8-row groups 1024 B apart), descriptor version 1.
 __device__ __forceinline__ uint64_t sw128_desc(const void *p)
@@ -95,8 +100,6 @@ __device__ __forceinline__ uint64_t sw128_desc(const void *p)
     d |= 2ull << 61;                          // 128-byte swizzle
     return d;
 }
-// Instruction descriptor, kind::f16: fp32 D, bf16 A and B, both K-major, M x N.
-
 // Instruction descriptor, kind::f16: fp32 D, bf16 A and B, both K-major, M x N.
 constexpr uint32_t idesc_bf16(int M, int N)
 {
@@ -123,6 +126,71 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
         "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
         : "memory");
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 16 fp32 registers into 16 consecutive columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15]))
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: MN-major operand in 128-byte-swizzled
+// atoms (each 128-byte row holds 64 consecutive M/N elements of one k; 8-row
+// k groups 1024 B apart), 64-element M/N blocks `lbo` bytes apart.
+__device__ __forceinline__ uint64_t sw128_mn_desc(const void *p, uint32_t lbo)
+{
+    const uint64_t addr = smem_addr(p);
+    uint64_t d = (addr >> 4) & 0x3FFFull;             // start address
+    d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;         // leading byte offset: next M/N block
+    d |= uint64_t(1024 >> 4) << 32;                    // stride byte offset: next 8 k rows
+    d |= 1ull << 46;                                   // version
+    d |= 2ull << 61;                                   // 128-byte swizzle
+    return d;
+}
+// Instruction descriptor as idesc_bf16 with A read MN-major (transposed).
+constexpr uint32_t idesc_bf16_amn(int M, int N) { return idesc_bf16(M, N) | (1u << 15); }
+
+// Per-thread 16-byte asynchronous copy global -> shared (L2 only), and the
+// mbarrier arrival that fires once all of this thread's earlier copies have
+// landed (counted against the barrier's expected arrivals).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // Generic-proxy shared-memory writes made visible to the async proxy (the
