@@ -209,10 +209,9 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
     };
     auto aborted = [&]() { return *(volatile int *)&abort_flag != 0; };
 
-    // V stages and P start at zero: rows of keys past a tile's end are read by
-    // the MMA with P = 0, so they must be finite.
-    for (int x = tid; x < 2 * kDtTile / 16; x += kDtThreads)
-        reinterpret_cast<uint4 *>(smem + Sm::oV)[x] = make_uint4(0u, 0u, 0u, 0u);
+    // P starts at zero (its rows past the query rows are never written).  V
+    // needs no clearing: P.V reads only the 16-key steps that hold keys of the
+    // tile, and the loads fill every row of those steps.
     for (int x = tid; x < 2 * kDtOpHalf / 16; x += kDtThreads)
         reinterpret_cast<uint4 *>(smem + Sm::oP)[x] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
@@ -256,7 +255,8 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                 tile_at(j, p0, n);
                 // every run of the window starts at a multiple of 8 rows, so
                 // the boxes cover roundup(n, 8) rows
-                mbar_arrive_expect_tx(&tfull[s], uint32_t((n + 7) / 8) * 8u * 512u);
+                const int ng = (n + 7) / 8;
+                mbar_arrive_expect_tx(&tfull[s], uint32_t(ng) * 8u * 512u + ((ng & 1) ? 8u * 256u : 0u));
                 uint8_t *kst = smem + Sm::oRaw + s * kDtTile, *vst = smem + Sm::oV + s * kDtTile;
                 for (int r = 0; r < n;) {
                     // the run holding window row p0 + r and that row's source
@@ -291,6 +291,12 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                         tma_load_2d(vst + r * 128, vm, 0, int(y), &tfull[s]);
                         tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), &tfull[s]);
                         r += dt_box_rows(hs);
+                        if (r >= n && (r & 8)) {
+                            // odd number of 8-row groups: one more box of the
+                            // same rows fills the tile's last 16-key step
+                            tma_load_2d(vst + r * 128, vm, 0, int(y), &tfull[s]);
+                            tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), &tfull[s]);
+                        }
                         y += dt_box_rows(hs);
                         len -= dt_box_rows(hs);
                     }
@@ -308,6 +314,13 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
             const uint32_t id_s = idesc_bf16(kDtKeys, kDtN), id_o = idesc_bf16_amn(D, kDtN);
             const uint8_t *kh = smem + Sm::oKh, *kl = smem + Sm::oKl, *qo = smem + Sm::oQ,
                           *po = smem + Sm::oP;
+            // operand descriptors at their k = 0 step
+            const uint64_t dKh[2] = {sw128_desc(kh), sw128_desc(kh + kDtHalf)};
+            const uint64_t dKl[2] = {sw128_desc(kl), sw128_desc(kl + kDtHalf)};
+            const uint64_t dQ[2] = {sw128_desc(qo), sw128_desc(qo + kDtOpHalf)};
+            const uint64_t dP0 = sw128_desc(po), dP1 = sw128_desc(po + kDtOpHalf);
+            const uint64_t dV0 = sw128_mn_desc(smem + Sm::oV, kDtHalf);
+            const uint64_t dV1 = sw128_mn_desc(smem + Sm::oV + kDtTile, kDtHalf);
             const bool qok = nt == 0 || (!aborted() && mbar_wait_bounded(qready, 0, kWaitLimitNs));
             if (!qok) fail();
             // S(js) as soon as tile js is converted (and its S buffer read),
@@ -324,11 +337,9 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const int bx = ks / 4, kin = ks % 4;
-                        const uint64_t ah = sw128_desc(kh + bx * kDtHalf) + uint64_t(kin * 2);
-                        const uint64_t al = sw128_desc(kl + bx * kDtHalf) + uint64_t(kin * 2);
-                        const uint64_t bq = sw128_desc(qo + bx * kDtOpHalf) + uint64_t(kin * 2);
-                        tc_mma(d_s, ah, bq, id_s, ks > 0 ? 1u : 0u);
-                        tc_mma(d_s, al, bq, id_s, 1u);
+                        tc_mma(d_s, dKh[bx] + uint64_t(kin * 2), dQ[bx] + uint64_t(kin * 2), id_s,
+                               ks > 0 ? 1u : 0u);
+                        tc_mma(d_s, dKl[bx] + uint64_t(kin * 2), dQ[bx] + uint64_t(kin * 2), id_s, 1u);
                     }
                     tc_commit(&sfull[s]);
                     tc_commit(kopempty);
@@ -338,13 +349,14 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                 if (jp < js && mbar_test(pfull, uint32_t(jp) & 1u) &&
                     mbar_test(&tfull[jp & 1], uint32_t(jp >> 1) & 1u)) {
                     const int s = jp & 1;
+                    int p0, n;
+                    tile_at(jp, p0, n);
                     tc_fence_after();
-                    const uint8_t *vt = smem + Sm::oV + s * kDtTile;
-#pragma unroll
-                    for (int ks = 0; ks < kDtKeys / 16; ++ks) {
-                        const uint64_t av = sw128_mn_desc(vt + ks * 2048, kDtHalf);
-                        const uint64_t bp = sw128_desc(po + (ks / 4) * kDtOpHalf) + uint64_t((ks % 4) * 2);
-                        tc_mma(tmem + 32u, av, bp, id_o, (jp > 0 || ks > 0) ? 1u : 0u);
+                    const uint64_t av0 = s ? dV1 : dV0;
+                    for (int ks = 0; ks < (n + 15) / 16; ++ks) {
+                        // 16 keys = 2048 bytes of V (descriptor units of 16 B)
+                        const uint64_t bp = (ks < 4 ? dP0 : dP1) + uint64_t((ks % 4) * 2);
+                        tc_mma(tmem + 32u, av0 + uint64_t(ks * 128), bp, id_o, (jp > 0 || ks > 0) ? 1u : 0u);
                     }
                     tc_commit(pvdone);
                     tc_commit(&vempty[s]);

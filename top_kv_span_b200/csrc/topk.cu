@@ -19,7 +19,10 @@ namespace reatt {
 
 namespace {
 
-constexpr int kTopkThreads = 512;
+#ifndef REATT_TOPK_THREADS
+#define REATT_TOPK_THREADS 512
+#endif
+constexpr int kTopkThreads = REATT_TOPK_THREADS;
 constexpr int kSlice = 4096;
 
 struct SelScratch {
@@ -124,11 +127,15 @@ __device__ void radix_select(Get get, int n, uint32_t kk, SelScratch &sc, uint32
 constexpr int kMaxE = 16;
 constexpr int kBins = 2048;
 
+constexpr int kWarpResolve = 32;   // candidates one warp ranks directly
+
 struct RegScratch {
     uint32_t hist[kBins];
     uint32_t red[2][32];
     int wsum[33];
-    uint32_t bcast[2];
+    uint32_t bcast[3];
+    uint32_t cand[kWarpResolve];
+    int ncand;
 };
 
 __device__ __forceinline__ void block_minmax(uint32_t mx, uint32_t mn, RegScratch &sc,
@@ -212,6 +219,8 @@ __device__ void select_regs(const uint32_t (&u)[E], int nvalid_mine, uint32_t kk
                 if (acc + c >= remaining) {
                     sc.bcast[0] = uint32_t(bin);
                     sc.bcast[1] = acc;
+                    sc.bcast[2] = c;   // codes left with the new prefix
+                    sc.ncand = 0;
                     break;
                 }
                 acc += c;
@@ -222,7 +231,36 @@ __device__ void select_regs(const uint32_t (&u)[E], int nvalid_mine, uint32_t kk
         prefix |= sc.bcast[0] << lo;
         mask |= dmask << lo;
         hb = lo - 1;
+        const uint32_t left = sc.bcast[2];
         __syncthreads();
+        if (hb >= 0 && left <= uint32_t(kWarpResolve)) {
+            // Few codes share the prefix: gather them and let one warp rank
+            // them (the remaining-th largest is tau).
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                if (e < nvalid_mine && (u[e] & mask) == prefix)
+                    sc.cand[atomicAdd(&sc.ncand, 1)] = u[e];
+            __syncthreads();
+            if (threadIdx.x < 32) {
+                const int lane = threadIdx.x, n = sc.ncand;
+                const uint32_t v = lane < n ? sc.cand[lane] : 0u;
+                uint32_t gt = 0, eq = 0;
+                for (int j = 0; j < n; ++j) {
+                    const uint32_t w = __shfl_sync(0xffffffffu, v, j);
+                    gt += w > v;
+                    eq += w == v;
+                }
+                if (lane < n && gt < remaining && remaining <= gt + eq) {
+                    sc.bcast[0] = v;                 // every such lane writes the same
+                    sc.bcast[1] = remaining - gt;
+                }
+            }
+            __syncthreads();
+            tau = sc.bcast[0];
+            take_eq = sc.bcast[1];
+            __syncthreads();
+            return;
+        }
     }
     tau = prefix;
     take_eq = remaining;
@@ -239,11 +277,13 @@ __device__ void compact_regs(const uint32_t (&u)[E], int nvalid_mine, uint32_t t
             n_gt += u[e] > tau;
             n_eq += u[e] == tau;
         }
+    // one scan of both counts (ties in the high half; totals stay below 2^16)
     int tot;
-    const int eq_before = block_exclusive_sum(n_eq, sc.wsum, &tot);
+    const int before = block_exclusive_sum((n_eq << 16) | n_gt, sc.wsum, &tot);
+    const int eq_before = before >> 16, gt_before = before & 0xffff;
     int take = int(take_eq) - eq_before;
     take = take < 0 ? 0 : (take > n_eq ? n_eq : take);
-    int pos = block_exclusive_sum(n_gt + take, sc.wsum, &tot);
+    int pos = gt_before + (eq_before < int(take_eq) ? eq_before : int(take_eq));
 #pragma unroll
     for (int e = 0; e < E; ++e)
         if (e < nvalid_mine) {
