@@ -86,14 +86,15 @@ __device__ __forceinline__ void split_range(const Geom &geo, int64_t W, int nspl
 // End of a CTA's work: its (max, sum, acc) per row sit in shared memory.  With
 // one split the output is written directly; otherwise the split's partial
 // goes to the workspace and the last CTA of (bh, qb) to finish (atomic ticket,
-// no waiting) merges all splits.  `scratch` holds >= nsplit*QB floats.
+// no waiting) merges all splits.  `scratch` holds >= 4 * 6 * nrows * D/4
+// floats when blockDim.x >= 2 * nrows * D/4 (shared memory of the caller).
 template <int D, int QB>
 __device__ void split_finish(const Geom &geo, const AttnArgs &a, int64_t bh, int qb, int split,
                              int nrows, const float *s_m, const float *s_l, const float *s_acc,
                              float *scratch, int *is_last)
 {
     constexpr int D4 = D / 4;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthr = blockDim.x;
+    const int tid = threadIdx.x, nthr = blockDim.x;
     const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv), r0 = qb * QB;
     auto out4 = [&](int rr) {
         const int r = r0 + rr, j = h * geo.g + r / geo.C, c = r % geo.C;
@@ -123,47 +124,69 @@ __device__ void split_finish(const Geom &geo, const AttnArgs &a, int64_t bh, int
     __syncthreads();
     if (!*is_last) return;
     __threadfence();
-    // w[s][r] = exp2(m_s - M_r) / sum_s' l_s' exp2(m_s' - M_r)
-    float *wgt = scratch;
+    // out = sum_s exp2(m_s - M) acc_s / sum_s exp2(m_s - M) l_s, merged online.
+    // With few output elements, G groups of threads take every G-th split of
+    // the same element (so all loads are in flight at once) and combine
+    // through `scratch` (G * items * 6 floats).
+    const int items = nrows * D4;
+    int G = nthr / items;
+    G = G < 1 ? 1 : (G > 4 ? 4 : G);
     const float2 *ml = a.part_ml + pbase * QB;
-    for (int x = tid; x < a.nsplit * QB; x += nthr) {
-        const int rr = x % QB;
-        wgt[x] = rr < nrows ? __ldcg(&ml[x].x) : -INFINITY;
-    }
-    __syncthreads();
-    for (int rr = warp; rr < nrows; rr += nthr / 32) {
-        float mx = -INFINITY;
-        for (int s = lane; s < a.nsplit; s += 32) mx = fmaxf(mx, wgt[s * QB + rr]);
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        float den = 0.f;
-        for (int s = lane; s < a.nsplit; s += 32) {
-            const float ms = wgt[s * QB + rr];
-            const float w = ms == -INFINITY ? 0.f : exp2f(ms - mx);
-            den += w * __ldcg(&ml[s * QB + rr].y);
-            wgt[s * QB + rr] = w;
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        const float iden = 1.f / den;
-        __syncwarp();
-        for (int s = lane; s < a.nsplit; s += 32) wgt[s * QB + rr] *= iden;
-    }
-    __syncthreads();
     const float4 *all = reinterpret_cast<const float4 *>(a.part_acc + pbase * int64_t(QB) * D);
-    for (int x = tid; x < nrows * D4; x += nthr) {
-        const int rr = x / D4;
+    auto fold = [&](float &M, float &den, float4 &z, float m, float l, float4 c) {
+        if (m == -INFINITY) return;
+        const float mn = fmaxf(M, m);
+        const float fo = M == -INFINITY ? 0.f : exp2f(M - mn), fn = exp2f(m - mn);
+        den = den * fo + fn * l;
+        z.x = z.x * fo + fn * c.x;
+        z.y = z.y * fo + fn * c.y;
+        z.z = z.z * fo + fn * c.z;
+        z.w = z.w * fo + fn * c.w;
+        M = mn;
+    };
+    for (int x0 = 0; x0 < items; x0 += nthr / G) {
+        const int x = x0 + tid % (nthr / G), g = tid / (nthr / G);
+        float M = -INFINITY, den = 0.f;
         float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int s = 0; s < a.nsplit; ++s) {
-            const float w = wgt[s * QB + rr];
-            const float4 v = __ldcg(all + int64_t(s) * QB * D4 + x);
-            z.x = fmaf(w, v.x, z.x);
-            z.y = fmaf(w, v.y, z.y);
-            z.z = fmaf(w, v.z, z.z);
-            z.w = fmaf(w, v.w, z.w);
+        if (x < items && g < G) {
+            const int rr = x / D4;
+            for (int s0 = g; s0 < a.nsplit; s0 += 8 * G) {
+                float2 v[8];
+                float4 c[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (s0 + u * G < a.nsplit) {
+                        v[u] = __ldcg(&ml[(s0 + u * G) * QB + rr]);
+                        c[u] = __ldcg(all + int64_t(s0 + u * G) * QB * D4 + x);
+                    }
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (s0 + u * G < a.nsplit) fold(M, den, z, v[u].x, v[u].y, c[u]);
+            }
         }
-        out4(rr)[x % D4] = z;
+        if (G > 1) {
+            float *sx = scratch + (size_t(g) * items + (x < items ? x : 0)) * 6;
+            if (x < items && g < G && g > 0) {
+                sx[0] = M;
+                sx[1] = den;
+                sx[2] = z.x;
+                sx[3] = z.y;
+                sx[4] = z.z;
+                sx[5] = z.w;
+            }
+            __syncthreads();
+            if (x < items && g == 0)
+                for (int g2 = 1; g2 < G; ++g2) {
+                    const float *o = scratch + (size_t(g2) * items + x) * 6;
+                    fold(M, den, z, o[0], o[1], make_float4(o[2], o[3], o[4], o[5]));
+                }
+            __syncthreads();
+        }
+        if (x < items && g == 0) {
+            const int rr = x / D4;
+            const float iden = 1.f / den;
+            out4(rr)[x % D4] = make_float4(z.x * iden, z.y * iden, z.z * iden, z.w * iden);
+        }
     }
     if (tid == 0) a.ticket[bh * a.nqb + qb] = 0u;   // ready for the next call
 }

@@ -11,14 +11,15 @@
 //   O^T (128 dims x 16) += V^T . [Ph ; Pl]^T         column r + column 8+r = O_r
 // Every rotated operand is split into bf16 hi + lo, so products keep fp32-level
 // accuracy (V is exact: bf16 input).  Roles of the 14 warps:
-//   warp 0      TMA: the tile's K and V rows in boxes of 8 rows x 64 columns,
-//               128B-swizzled (each box lies inside one run of the window: the
-//               global part, a chosen span, the local part, the current
-//               tokens); V lands directly in the MN-major operand layout
+//   warp 0      TMA: the tile's K and V rows in boxes of 32 or 8 rows x 64
+//               columns, 128B-swizzled, each inside one run of the window (the
+//               global part, a chosen span, the local part, the current tokens)
+//               and one 32-row quarter of the tile, which has its own barrier;
+//               V lands directly in the MN-major operand layout
 //   warp 1      TMEM allocation; one thread issues S(j) and then P(j-1).V(j-1)
-//   warps 2-9   rotate the raw keys (RoPE, angle anchored from the step's table
-//               every 4 keys and advanced by the one-position rotation), split
-//               them into the hi/lo K-major operands
+//   warps 2-9   rotate the raw keys of each quarter as it lands (RoPE with
+//               the step's cos/sin table) and split them into the hi/lo
+//               K-major operands
 //   warps 10-13 the rotated query operand first; then softmax: thread t owns
 //               key t of the tile (TMEM lane t): online
 //               softmax with a lazily moved reference max (rescales O in TMEM
@@ -52,11 +53,9 @@ constexpr int kDtThreads = (kDtSoftBase + kDtSoftWarps) * 32;
 constexpr int kDtHalf = kDtKeys * 128;                // 64-column half of a tile: 16 KB
 constexpr int kDtTile = 2 * kDtHalf;                  // 128 rows x 128 bf16
 constexpr int kDtOpHalf = kDtN * 128;                 // half of the 16-row Q / P operands
-constexpr int kDtKeysPerConv = kDtKeys * 8 / (kDtConvWarps * 32);   // 4 keys per thread
 constexpr uint32_t kDtTmemCols = 64;                  // S buffers at 0 and 16, O at 32
 constexpr float kDtRescaleLog2 = 8.f;
 constexpr int kDtSelCache = 256;                      // chosen span ids of a CTA's rows
-static_assert(kDtKeysPerConv * kDtConvWarps * 32 == kDtKeys * 8, "converter map");
 static_assert(kDtSoftWarps * 32 == kDtKeys, "one softmax thread per key");
 
 // Shared memory (1024-byte aligned): raw K stages | V stages | Kh | Kl | Q | P |
@@ -94,12 +93,13 @@ __device__ __forceinline__ void split_pack(float a, float b, uint32_t &hi, uint3
     lo = pack_bf16(a - ha, b - hb);
 }
 
-// Tensor maps of the caches (boxes of 128, 32 and 8 rows) and of the current
+// Tensor maps of the caches (boxes of 32 and 8 rows) and of the current
 // tokens (8 rows); every box is 64 columns wide.
 struct DtMaps {
-    CUtensorMap k[3], v[3], kq, vq;
+    CUtensorMap k[2], v[2], kq, vq;
 };
-__host__ __device__ constexpr int dt_box_rows(int i) { return i == 0 ? 128 : (i == 1 ? 32 : 8); }
+__host__ __device__ constexpr int dt_box_rows(int i) { return i == 0 ? 32 : 8; }
+constexpr int kDtQuarter = 32;                        // rows per load barrier
 
 template <int RP>
 __global__ void __launch_bounds__(kDtThreads, 1)
@@ -111,10 +111,12 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Sm::oBar);
-    uint64_t *tfull = bars, *rawempty = bars + 2, *vempty = bars + 4, *kopfull = bars + 6,
+    uint64_t *rawempty = bars + 2, *vempty = bars + 4, *kopfull = bars + 6,
              *kopempty = bars + 7, *sfull = bars + 8, *sempty = bars + 10, *pfull = bars + 12,
              *pvdone = bars + 13, *done = bars + 14, *qready = bars + 15;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+    // loads of stage s, rows [32q, 32q + 32): tq[4s + q]
+    uint64_t *tq = bars + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 24);
     __shared__ float red[2][kDtSoftWarps][RP], lred[kDtSoftWarps][RP];
     __shared__ float f_m[RP], f_l[RP];
     __shared__ __align__(16) float s_acc[RP * D];
@@ -126,7 +128,6 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
     if (tid == 0) {
         abort_flag = 0;
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&tfull[s], 1);
             mbar_init(&rawempty[s], kDtConvWarps);
             mbar_init(&vempty[s], 1);
             mbar_init(&sfull[s], 1);
@@ -138,6 +139,7 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
         mbar_init(pvdone, 1);
         mbar_init(done, 1);
         mbar_init(qready, kDtSoftWarps);
+        for (int q = 0; q < 8; ++q) mbar_init(&tq[q], 1);
         mbar_init_fence();
     }
     if (warp == 1) {
@@ -223,7 +225,7 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
     if (warp == 0) {
         // ------------------------------------------------ loads (TMA)
         if (lane == 0)
-            for (int i = 0; i < 3; ++i) {
+            for (int i = 0; i < 2; ++i) {
                 prefetch_tensormap(&maps.k[i]);
                 prefetch_tensormap(&maps.v[i]);
             }
@@ -255,8 +257,19 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                 tile_at(j, p0, n);
                 // every run of the window starts at a multiple of 8 rows, so
                 // the boxes cover roundup(n, 8) rows
+                // bytes per 32-row quarter: K and V rows (both halves), plus
+                // the V pad box of an odd last group; one arrival each
                 const int ng = (n + 7) / 8;
-                mbar_arrive_expect_tx(&tfull[s], uint32_t(ng) * 8u * 512u + ((ng & 1) ? 8u * 256u : 0u));
+                for (int q = 0; q < 4; ++q) {
+                    int rows = 8 * ng - kDtQuarter * q;
+                    rows = rows < 0 ? 0 : (rows > kDtQuarter ? kDtQuarter : rows);
+                    uint32_t bytes = uint32_t(rows) * 512u;
+                    if ((ng & 1) && (8 * ng) / kDtQuarter == q) bytes += 8u * 256u;
+                    if (bytes)
+                        mbar_arrive_expect_tx(&tq[4 * s + q], bytes);
+                    else
+                        mbar_arrive(&tq[4 * s + q]);
+                }
                 uint8_t *kst = smem + Sm::oRaw + s * kDtTile, *vst = smem + Sm::oV + s * kDtTile;
                 for (int r = 0; r < n;) {
                     // the run holding window row p0 + r and that row's source
@@ -283,19 +296,22 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                     }
                     int len = (run_end < p0 + n ? run_end : p0 + n) - p;
                     while (len > 0) {
-                        const int hs = cur ? 2 : (len >= 128 ? 0 : (len >= 32 ? 1 : 2));
+                        // 32-row boxes start on a quarter, so none crosses one
+                        const int hs = (!cur && len >= 32 && (r & 31) == 0) ? 0 : 1;
                         const CUtensorMap *km = cur ? &maps.kq : &maps.k[hs];
                         const CUtensorMap *vm = cur ? &maps.vq : &maps.v[hs];
-                        tma_load_2d(kst + r * 128, km, 0, int(y), &tfull[s]);
-                        tma_load_2d(kst + kDtHalf + r * 128, km, 64, int(y), &tfull[s]);
-                        tma_load_2d(vst + r * 128, vm, 0, int(y), &tfull[s]);
-                        tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), &tfull[s]);
+                        uint64_t *bar = &tq[4 * s + r / kDtQuarter];
+                        tma_load_2d(kst + r * 128, km, 0, int(y), bar);
+                        tma_load_2d(kst + kDtHalf + r * 128, km, 64, int(y), bar);
+                        tma_load_2d(vst + r * 128, vm, 0, int(y), bar);
+                        tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), bar);
                         r += dt_box_rows(hs);
                         if (r >= n && (r & 8)) {
                             // odd number of 8-row groups: one more box of the
                             // same rows fills the tile's last 16-key step
-                            tma_load_2d(vst + r * 128, vm, 0, int(y), &tfull[s]);
-                            tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), &tfull[s]);
+                            uint64_t *pbar = &tq[4 * s + r / kDtQuarter];
+                            tma_load_2d(vst + r * 128, vm, 0, int(y), pbar);
+                            tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), pbar);
                         }
                         y += dt_box_rows(hs);
                         len -= dt_box_rows(hs);
@@ -306,8 +322,10 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
         }
         // drain: the last loads of each stage have landed
         for (int j = nt - 2 < 0 ? 0 : nt - 2; ok && j < nt; ++j)
-            if (!mbar_wait_bounded(&tfull[j & 1], uint32_t(j >> 1) & 1u, kWaitLimitNs) && lane == 0)
-                fail();
+            for (int q = 0; q < 4; ++q)
+                if (!mbar_wait_bounded(&tq[4 * (j & 1) + q], uint32_t(j >> 1) & 1u, kWaitLimitNs) &&
+                    lane == 0)
+                    fail();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -347,7 +365,10 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                     progressed = true;
                 }
                 if (jp < js && mbar_test(pfull, uint32_t(jp) & 1u) &&
-                    mbar_test(&tfull[jp & 1], uint32_t(jp >> 1) & 1u)) {
+                    mbar_test(&tq[4 * (jp & 1)], uint32_t(jp >> 1) & 1u) &&
+                    mbar_test(&tq[4 * (jp & 1) + 1], uint32_t(jp >> 1) & 1u) &&
+                    mbar_test(&tq[4 * (jp & 1) + 2], uint32_t(jp >> 1) & 1u) &&
+                    mbar_test(&tq[4 * (jp & 1) + 3], uint32_t(jp >> 1) & 1u)) {
                     const int s = jp & 1;
                     int p0, n;
                     tile_at(jp, p0, n);
@@ -368,6 +389,8 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                 } else if (aborted() || global_ns() - t_last > kWaitLimitNs) {
                     fail();
                     break;
+                } else {
+                    __nanosleep(64);   // leave the issue slots to the working warps
                 }
             }
             tc_commit(done);
@@ -376,22 +399,20 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
         __syncwarp();   // idle lanes wait here, not in the grid-dependency wait below
     } else if (warp < kDtSoftBase) {
         // ------------------------------------------------ RoPE + hi/lo split of K
+        // All converter warps take each 32-row quarter as soon as it lands:
+        // thread = (key kq of the quarter, pair chunk c); the key's cos/sin
+        // come from the step's table, loaded one quarter ahead.
         const int ct = tid - kDtConvBase * 32;
         const int c = ct & 7;                    // pairs 8c..8c+7 (dims and dims + 64)
-        const int k0 = (ct >> 3) * kDtKeysPerConv;
-        float2 st[8];                             // one-position rotation per frequency
-#pragma unroll
-        for (int e = 0; e < 8; ++e) rope_cs(1, freq[8 * c + e].x, freq[8 * c + e].y, st[e].x, st[e].y);
-        // cos/sin at this thread's first key of tile j, from the step's table
-        // (loaded one tile ahead)
-        auto anchors = [&](int j, float2 (&cs)[8]) {
+        const int kq = ct >> 3;                  // 0..31
+        static_assert(kDtConvWarps * 32 == kDtQuarter * 8, "one (key, chunk) per thread and quarter");
+        auto anchors = [&](int job, float2 (&cs)[8]) {
+            const int j = job >> 2, r = kDtQuarter * (job & 3) + kq;
             int p0, n;
             tile_at(j, p0, n);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) cs[e] = make_float2(1.f, 0.f);
-            if (k0 < n) {
+            if (r < n) {
                 const float4 *tr =
-                    reinterpret_cast<const float4 *>(a.tab + int64_t(p0 + k0) * (D / 2) + 8 * c);
+                    reinterpret_cast<const float4 *>(a.tab + int64_t(p0 + r) * (D / 2) + 8 * c);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float4 t = __ldcg(tr + e);
@@ -401,28 +422,31 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
             }
         };
         float2 nx[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) nx[e] = make_float2(1.f, 0.f);
         if (nt > 0) anchors(0, nx);
         bool ok = true;
-        for (int j = 0; j < nt; ++j) {
+        uint8_t *kh = smem + Sm::oKh, *kl = smem + Sm::oKl;
+        for (int j = 0; j < nt && ok; ++j) {
             const int s = j & 1;
             int p0, n;
             tile_at(j, p0, n);
-            float2 cs[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) cs[e] = nx[e];
-            if (j + 1 < nt) anchors(j + 1, nx);
-            ok = ok && !aborted() &&
-                 mbar_wait_bounded(&tfull[s], uint32_t(j >> 1) & 1u, kWaitLimitNs) &&
-                 (j == 0 || mbar_wait_bounded(kopempty, uint32_t(j - 1) & 1u, kWaitLimitNs));
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) fail();
-                break;
-            }
             const uint8_t *raw = smem + Sm::oRaw + s * kDtTile;
-            uint8_t *kh = smem + Sm::oKh, *kl = smem + Sm::oKl;
+            for (int qd = 0; qd < 4; ++qd) {
+                float2 cs[8];
 #pragma unroll
-            for (int t = 0; t < kDtKeysPerConv; ++t) {
-                const int r = k0 + t;
+                for (int e = 0; e < 8; ++e) cs[e] = nx[e];
+                const int job = 4 * j + qd;
+                if (job + 1 < 4 * nt) anchors(job + 1, nx);
+                ok = ok && !aborted() &&
+                     mbar_wait_bounded(&tq[4 * s + qd], uint32_t(j >> 1) & 1u, kWaitLimitNs) &&
+                     (qd > 0 || j == 0 || mbar_wait_bounded(kopempty, uint32_t(j - 1) & 1u, kWaitLimitNs));
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0) fail();
+                    ok = false;
+                    break;
+                }
+                const int r = kDtQuarter * qd + kq;
                 if (r < n) {
                     const uint4 xw = *reinterpret_cast<const uint4 *>(raw + sw_off(r, c, kDtHalf));
                     const uint4 yw = *reinterpret_cast<const uint4 *>(raw + sw_off(r, c + 8, kDtHalf));
@@ -441,13 +465,8 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                     *reinterpret_cast<uint4 *>(kl + sw_off(r, c, kDtHalf)) = make_uint4(xl[0], xl[1], xl[2], xl[3]);
                     *reinterpret_cast<uint4 *>(kl + sw_off(r, c + 8, kDtHalf)) = make_uint4(yl[0], yl[1], yl[2], yl[3]);
                 }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {   // advance one position
-                    const float cn = cs[e].x * st[e].x - cs[e].y * st[e].y;
-                    cs[e].y = cs[e].y * st[e].x + cs[e].x * st[e].y;
-                    cs[e].x = cn;
-                }
             }
+            if (!ok) break;
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -638,7 +657,7 @@ cudaError_t launch_attend_decode_tc(const Geom &geo, const AttnArgs &a, int RP, 
     const bool has_cache = geo.T > 0;
     const void *kb = has_cache ? kc : kcur, *vb = has_cache ? vc : vcur;
     const uint64_t rows = has_cache ? BH * geo.T : BH * geo.C;
-    for (int i = 0; i < 3; ++i)
+    for (int i = 0; i < 2; ++i)
         if (!encode_bf16_map(&mp.k[i], kb, rows, kDtD, uint32_t(dt_box_rows(i))) ||
             !encode_bf16_map(&mp.v[i], vb, rows, kDtD, uint32_t(dt_box_rows(i))))
             return cudaErrorInvalidValue;
