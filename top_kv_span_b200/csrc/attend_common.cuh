@@ -115,15 +115,21 @@ __device__ void split_finish(const Geom &geo, const AttnArgs &a, int64_t bh, int
         pacc[x] = reinterpret_cast<const float4 *>(s_acc)[x];
     for (int rr = tid; rr < nrows; rr += nthr)
         a.part_ml[(pbase + split) * QB + rr] = make_float2(s_m[rr], s_l[rr]);
-    __threadfence();
+    // The barrier makes the CTA's partial writes precede thread 0's ticket
+    // increment, whose gpu-scope release publishes them (cumulatively); the
+    // last CTA's acquire on the same atomic makes every split's partial
+    // visible to it.
     __syncthreads();
     if (tid == 0) {
-        const uint32_t prev = atomicAdd(&a.ticket[bh * a.nqb + qb], 1u);
+        uint32_t prev;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(prev)
+                     : "l"(&a.ticket[bh * a.nqb + qb])
+                     : "memory");
         *is_last = prev == uint32_t(a.nsplit - 1);
     }
     __syncthreads();
     if (!*is_last) return;
-    __threadfence();
     // out = sum_s exp2(m_s - M) acc_s / sum_s exp2(m_s - M) l_s, merged online.
     // With few output elements, G groups of threads take every G-th split of
     // the same element (so all loads are in flight at once) and combine
