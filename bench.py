@@ -143,6 +143,13 @@ def aggregate(world, step_b, steps, total_ms, e2e_ms, scan_ms, reduce_max=None):
             "e2e_value": world * step_b * steps / (e2e_ms * 1e-3) / 1e9}
 
 
+def dist_us(ms_list):
+    """Median, p10 and p90 (µs) of a list of per-step times in ms."""
+    v = sorted(ms_list)
+    pick = lambda f: v[min(len(v) - 1, int(round(f * (len(v) - 1))))] * 1e3
+    return {"median": round(pick(0.5), 2), "p10": round(pick(0.1), 2), "p90": round(pick(0.9), 2)}
+
+
 def peaks():
     """(HBM GB/s, bf16 TFLOP/s burst, kind): the measured copy bandwidth and
     cuBLAS bf16 throughput of this machine's B200s, else the earlier fallback."""
@@ -269,7 +276,8 @@ def run_ours(args):
         scan_only()
         sev[i][1].record(stream)
     torch.cuda.synchronize(dev)
-    scan_ms = statistics.mean(a.elapsed_time(b) for a, b in sev)
+    scan_list = [a.elapsed_time(b) for a, b in sev]
+    scan_ms = statistics.mean(scan_list)
 
     # end to end through the C ABI with host buffers: per step the new
     # token's q / k / v go host->device from pinned memory and the output
@@ -335,6 +343,9 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms / args.steps * 1e3, 2)},
         "gpu_launches": per_step * args.steps,
         "clocks": clk.summary(),
+        # this rank's distribution over the timed steps (µs): median, p10, p90
+        "step_dist_us": dist_us(step_ms),
+        "scan_dist_us": dist_us(scan_list),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, x, seconds=args.cpu_seconds)

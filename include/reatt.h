@@ -93,6 +93,9 @@ typedef struct {
     int32_t dtype;      /* reatt_dtype of q, caches and current tokens         */
     int64_t T;          /* cached tokens, 0 <= T < 2^31                         */
     double rope_base;   /* RoPE base (> 0, finite)                              */
+    int64_t T_cap;      /* rows allocated per (batch, KV head) in k_cache and
+                           v_cache: row t of (b, h) is at ((b*Hkv + h)*T_cap + t)*d;
+                           0 means T (dense caches); otherwise T <= T_cap < 2^31 */
 } reatt_dims;
 
 /* Text for a status code (static storage; never NULL). */
@@ -170,6 +173,19 @@ REATT_API int reatt_attend(const reatt_dims *dims, const void *q, const float *k
 REATT_API int reatt_step(const reatt_dims *dims, const void *q, const void *k_cache, const void *v_cache,
                const void *k_cur, const void *v_cur, int32_t *sel_out, float *out, void *ws,
                reatt_stream stream);
+
+/*
+ * Appends the C current tokens' K and V rows to the caches (the caller's step
+ * after each reatt_step of a decoding loop or a chunked prefill; the pages'
+ * prefilling and decoding pseudocode add the new keys and values to the cache
+ * after the attention, ReAttention OpenReview discussion):
+ *   k_cache[b,h,T+c,:] = k_cur[b,h,c,:], same for v, for c < C,
+ * with cache rows at stride T_cap (dims->T_cap >= T + C, else EINVAL).
+ * k_cur, v_cur [B,Hkv,C,d] in dims->dtype; all pointers 16-byte aligned.
+ * The next call then uses dims with T + C.
+ */
+REATT_API int reatt_append_kv(const reatt_dims *dims, void *k_cache, void *v_cache,
+                              const void *k_cur, const void *v_cur, reatt_stream stream);
 
 /*
  * Diagnostic for the failure-detection path: launches one thread that waits

@@ -32,9 +32,31 @@ def test_exports_every_declared_symbol(R):
 
 
 def test_dims_struct_layout_matches_header(R):
-    # int32 x 10, int64, double -> 56 bytes, T at offset 40
-    assert ctypes.sizeof(R.reatt_dims) == 56
+    # int32 x 10, int64 T, double rope_base, int64 T_cap -> 64 bytes
+    assert ctypes.sizeof(R.reatt_dims) == 64
     assert R.reatt_dims.T.offset == 40 and R.reatt_dims.rope_base.offset == 48
+    assert R.reatt_dims.T_cap.offset == 56
+
+
+def test_cache_capacity_checks(R):
+    # T_cap below T is rejected everywhere; 0 means dense caches (T rows)
+    nbytes = ctypes.c_size_t()
+    bad = R.make_dims(B=1, Hq=8, Hkv=2, d=128, C=1, T=1000, G=4, L=16, S=8, k=4, dtype="bf16",
+                      rope_base=1e4, T_cap=999)
+    assert R.lib.reatt_workspace_bytes(ctypes.byref(bad), ctypes.byref(nbytes)) == R.EINVAL
+    ok = R.make_dims(B=1, Hq=8, Hkv=2, d=128, C=1, T=1000, G=4, L=16, S=8, k=4, dtype="bf16",
+                     rope_base=1e4, T_cap=4096)
+    assert R.lib.reatt_workspace_bytes(ctypes.byref(ok), ctypes.byref(nbytes)) == R.OK
+    # appending needs room for C rows past T, and every pointer
+    dense = R.make_dims(B=1, Hq=8, Hkv=2, d=128, C=1, T=1000, G=4, L=16, S=8, k=4, dtype="bf16",
+                        rope_base=1e4)
+    fake = 1 << 20   # never dereferenced: the checks fail first
+    assert R.reatt_append_kv(dense, fake, fake, fake, fake, stream=0, check=False) == R.EINVAL
+    full = R.make_dims(B=1, Hq=8, Hkv=2, d=128, C=2, T=1000, G=4, L=16, S=8, k=4, dtype="bf16",
+                       rope_base=1e4, T_cap=1001)
+    assert R.reatt_append_kv(full, fake, fake, fake, fake, stream=0, check=False) == R.EINVAL
+    assert R.reatt_append_kv(ok, None, fake, fake, fake, stream=0, check=False) == R.EINVAL
+    assert R.reatt_append_kv(ok, fake + 8, fake, fake, fake, stream=0, check=False) == R.EINVAL
 
 
 def test_status_strings(R):

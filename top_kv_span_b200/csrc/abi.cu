@@ -25,10 +25,11 @@ int make_geom(const reatt_dims *d, Geom *g)
     if (d->d != 64 && d->d != 128) return REATT_EUNSUPPORTED;
     if (d->k > 65536) return REATT_EUNSUPPORTED;
     if (d->T >= (int64_t(1) << 31)) return REATT_EUNSUPPORTED;
+    if (d->T_cap != 0 && (d->T_cap < d->T || d->T_cap >= (int64_t(1) << 31))) return REATT_EINVAL;
     const double wmax = double(d->G) + double(d->k) * d->S + d->L + d->C;
     if (wmax >= 2147483647.0) return REATT_EUNSUPPORTED;
     // element counts of the largest buffers must fit comfortably in int64
-    const double cache = double(d->B) * d->Hkv * double(d->T) * d->d;
+    const double cache = double(d->B) * d->Hkv * double(d->T_cap ? d->T_cap : d->T) * d->d;
     const double win = double(d->B) * d->Hkv * wmax * d->d;
     const double qn = double(d->B) * d->Hq * double(d->C) * d->d;
     if (cache > 4e18 || win > 4e18 || qn > 4e18) return REATT_EUNSUPPORTED;
@@ -44,6 +45,7 @@ int make_geom(const reatt_dims *d, Geom *g)
     g->S = d->S;
     g->k = d->k;
     g->T = d->T;
+    g->Ts = d->T_cap ? d->T_cap : d->T;
     g->g_end = d->T < d->G ? d->T : d->G;
     g->loc_begin = (d->T - d->L) > d->G ? (d->T - d->L) : d->G;
     g->n_loc = d->T > g->loc_begin ? d->T - g->loc_begin : 0;
@@ -267,6 +269,20 @@ int reatt_step(const reatt_dims *dims, const void *q, const void *k_cache, const
     return cuda_status(launch_attend(g, q, nullptr, nullptr, nullptr, k_cache, v_cache, k_cur,
                                      v_cur, sel, tab, out, at(ws, p.ticket), ws, true, st,
                                      w_known));
+}
+
+int reatt_append_kv(const reatt_dims *dims, void *k_cache, void *v_cache, const void *k_cur,
+                    const void *v_cur, reatt_stream stream)
+{
+    Geom g;
+    const int rc = make_geom(dims, &g);
+    if (rc) return rc;
+    if (g.Ts < g.T + g.C) return REATT_EINVAL;   // the caches have no room for C more rows
+    if (!k_cache || !v_cache || !k_cur || !v_cur) return REATT_EINVAL;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_cur) || !aligned16(v_cur))
+        return REATT_EINVAL;
+    return cuda_status(launch_append(g, k_cache, v_cache, k_cur, v_cur,
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

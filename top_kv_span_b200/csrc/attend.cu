@@ -63,8 +63,8 @@ gather_rope_kernel(Geom geo, const T *__restrict__ kc, const T *__restrict__ vc,
         const int64_t s = win_src(geo, m, sel_bh, p);
         const T *kr, *vr;
         if (s >= 0) {
-            kr = kc + (bh * geo.T + s) * D;
-            vr = vc + (bh * geo.T + s) * D;
+            kr = kc + (bh * geo.Ts + s) * D;
+            vr = vc + (bh * geo.Ts + s) * D;
         } else {
             kr = kcur + (bh * geo.C + (-s - 1)) * D;
             vr = vcur + (bh * geo.C + (-s - 1)) * D;
@@ -168,7 +168,7 @@ __device__ __forceinline__ int64_t win_row_offset(const Geom &geo, const WinMap 
         const int c = p - g_end - nsel - nloc;
         return (int64_t(1) << 62) | ((bh * geo.C + c) * D);
     }
-    return (bh * geo.T + s) * D;
+    return (bh * geo.Ts + s) * D;
 }
 
 constexpr int kDecWarps = 8;
@@ -575,16 +575,16 @@ attend_staged_kernel(Geom geo, AttnArgs a, const T *__restrict__ kc, const T *__
                     bool cur = false;
                     int64_t o;
                     if (p < g_end) {
-                        o = (bh * geo.T + p) * D;
+                        o = (bh * geo.Ts + p) * D;
                     } else if (p - g_end < nsel) {
                         const int q = p - g_end, j = q / geo.S, off = q - j * geo.S;
                         int sp = sel_cached ? sel_s[j - j0] : sel_bh[j];
                         sp = sp < 0 ? 0 : (sp >= int(geo.NS) ? int(geo.NS) - 1 : sp);
                         int srow = geo.G + sp * geo.S + off;
                         if (srow >= int(geo.T)) srow = int(geo.T) - 1;
-                        o = (bh * geo.T + srow) * D;
+                        o = (bh * geo.Ts + srow) * D;
                     } else if (p - g_end - nsel < nloc) {
-                        o = (bh * geo.T + m.loc_begin + (p - g_end - nsel)) * D;
+                        o = (bh * geo.Ts + m.loc_begin + (p - g_end - nsel)) * D;
                     } else {
                         cur = true;
                         o = (bh * geo.C + (p - g_end - nsel - nloc)) * D;
@@ -852,8 +852,8 @@ struct KvSource<T, D, true> {
         const int64_t s = win_src(geo, m, sel_bh, p);
         const T *kr, *vr;
         if (s >= 0) {
-            kr = kc + (bh * geo.T + s) * D;
-            vr = vc + (bh * geo.T + s) * D;
+            kr = kc + (bh * geo.Ts + s) * D;
+            vr = vc + (bh * geo.Ts + s) * D;
         } else {
             kr = kcur + (bh * geo.C + (-s - 1)) * D;
             vr = vcur + (bh * geo.C + (-s - 1)) * D;

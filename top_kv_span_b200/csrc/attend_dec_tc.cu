@@ -279,16 +279,16 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                     int64_t y;
                     if (p < g_end) {
                         run_end = g_end;
-                        y = bh * geo.T + p;
+                        y = bh * geo.Ts + p;
                     } else if (p - g_end < nsel) {
                         const int q = p - g_end, jj = q / geo.S, off = q - jj * geo.S;
                         int sp = sel_cached ? sel_s[jj - j0] : sel_bh[jj];
                         sp = sp < 0 ? 0 : (sp >= int(geo.NS) ? int(geo.NS) - 1 : sp);
                         run_end = g_end + (jj + 1) * geo.S;
-                        y = bh * geo.T + geo.G + int64_t(sp) * geo.S + off;
+                        y = bh * geo.Ts + geo.G + int64_t(sp) * geo.S + off;
                     } else if (p - g_end - nsel < nloc) {
                         run_end = g_end + nsel + nloc;
-                        y = bh * geo.T + m.loc_begin + (p - g_end - nsel);
+                        y = bh * geo.Ts + m.loc_begin + (p - g_end - nsel);
                     } else {
                         run_end = int(W);
                         cur = true;
@@ -642,7 +642,7 @@ bool decode_tc_eligible(const Geom &geo)
     const int64_t BH = int64_t(geo.B) * geo.Hkv;
     return geo.dtype == REATT_BF16 && geo.d == kDtD && int64_t(geo.g) * geo.C <= 8 &&
            geo.g_end % 8 == 0 && geo.S % 8 == 0 && geo.n_loc % 8 == 0 &&
-           (geo.NS == 0 || geo.M % geo.S == 0) && BH * geo.T + 8 < (int64_t(1) << 31) &&
+           (geo.NS == 0 || geo.M % geo.S == 0) && BH * geo.Ts + 8 < (int64_t(1) << 31) &&
            BH * geo.C + 8 < (int64_t(1) << 31);
 }
 
@@ -656,7 +656,7 @@ cudaError_t launch_attend_decode_tc(const Geom &geo, const AttnArgs &a, int RP, 
     // an empty cache still needs valid maps: point them at the current tokens
     const bool has_cache = geo.T > 0;
     const void *kb = has_cache ? kc : kcur, *vb = has_cache ? vc : vcur;
-    const uint64_t rows = has_cache ? BH * geo.T : BH * geo.C;
+    const uint64_t rows = has_cache ? BH * geo.Ts : BH * geo.C;
     for (int i = 0; i < 2; ++i)
         if (!encode_bf16_map(&mp.k[i], kb, rows, kDtD, uint32_t(dt_box_rows(i))) ||
             !encode_bf16_map(&mp.v[i], vb, rows, kDtD, uint32_t(dt_box_rows(i))))

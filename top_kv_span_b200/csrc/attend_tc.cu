@@ -68,7 +68,7 @@ __device__ __forceinline__ WinMapTc winmap_tc(const Geom &geo, const int32_t *se
 __device__ __forceinline__ int64_t row_src_tc(const Geom &geo, const WinMapTc &m,
                                               const int32_t *sel_bh, int64_t bh, int64_t p, int D)
 {
-    if (p < m.g_end) return (bh * geo.T + p) * D;
+    if (p < m.g_end) return (bh * geo.Ts + p) * D;
     p -= m.g_end;
     if (p < m.nsel_rows) {
         const int64_t j = p / geo.S, off = p - j * geo.S;
@@ -76,10 +76,10 @@ __device__ __forceinline__ int64_t row_src_tc(const Geom &geo, const WinMapTc &m
         sp = sp < 0 ? 0 : (sp >= geo.NS ? geo.NS - 1 : sp);
         int64_t row = geo.G + sp * geo.S + off;
         if (row >= geo.T) row = geo.T - 1;
-        return (bh * geo.T + row) * D;
+        return (bh * geo.Ts + row) * D;
     }
     p -= m.nsel_rows;
-    if (p < m.n_loc) return (bh * geo.T + m.loc_begin + p) * D;
+    if (p < m.n_loc) return (bh * geo.Ts + m.loc_begin + p) * D;
     return (int64_t(1) << 62) | ((bh * geo.C + (p - m.n_loc)) * D);
 }
 

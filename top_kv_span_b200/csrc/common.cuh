@@ -13,6 +13,7 @@ namespace reatt {
 struct Geom {
     int B, Hq, Hkv, g, d, C, G, L, S, k;
     int64_t T;
+    int64_t Ts;         // cache rows per (b, KV head): T_cap, or T for dense caches
     int64_t g_end;      // min(G, T)
     int64_t loc_begin;  // max(G, T - L)
     int64_t n_loc;      // T - loc_begin if T > loc_begin else 0

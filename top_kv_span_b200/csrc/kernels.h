@@ -64,6 +64,10 @@ int topk_selecting_ctas(const Geom &geo);   // CTAs of the first top-k launch th
 cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void *scratch,
                         uint32_t *zero_words, int nzero, float2 *rope_tab, cudaStream_t st);
 
+// current tokens' K/V rows -> cache rows [T, T + C) (caches of Ts rows per head)
+cudaError_t launch_append(const Geom &geo, void *k_cache, void *v_cache, const void *k_cur,
+                          const void *v_cur, cudaStream_t st);
+
 cudaError_t launch_gather_rope(const Geom &geo, const void *kc, const void *vc, const void *kcur,
                                const void *vcur, const int32_t *sel, float *kw, float *vw,
                                int32_t *win_len, cudaStream_t st);

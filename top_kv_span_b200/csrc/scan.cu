@@ -161,7 +161,7 @@ scan_decode_kernel(Geom geo, const T *__restrict__ q, const T *__restrict__ kc,
             Item it;
             bool stop = false;
             while (!stop && next_item(geo, gs, cta_end, it)) {
-                const T *src = kc + (it.bh * geo.T + it.t_begin) * D;
+                const T *src = kc + (it.bh * geo.Ts + it.t_begin) * D;
                 for (int64_t t = it.t_begin; t < it.t_end; t += kStageTok, src += kStageTok * D) {
                     if (wrapped) {
                         if (*(volatile int *)&abort_flag ||
@@ -370,7 +370,7 @@ scan_multi_kernel(Geom geo, const float *__restrict__ qsum, const T *__restrict_
     if (t_end > geo.G + geo.M) t_end = geo.G + geo.M;
     for (int s = tid; s < kMqTile; s += 256) smax[s] = 0u;
     const float *qb = qsum + bh * int64_t(geo.C) * D;
-    const T *kb = kc + bh * geo.T * D;
+    const T *kb = kc + bh * geo.Ts * D;
 
     for (int64_t t0 = t_begin; t0 < t_end; t0 += kMqTile) {
         const int ntok = int(t_end - t0 < kMqTile ? t_end - t0 : kMqTile);

@@ -113,7 +113,7 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             for (int64_t it = blockIdx.x; ok && it < ta.items; it += gridDim.x) {
                 const int64_t bh = it / ta.ntiles;
                 const int tile = int(it % ta.ntiles);
-                const int y = int(bh * geo.T + geo.G + int64_t(tile) * kTiles * kTileM);
+                const int y = int(bh * geo.Ts + geo.G + int64_t(tile) * kTiles * kTileM);
                 if (kuse > 0 && (aborted() || !mbar_wait_bounded(kempty, (kuse - 1) & 1, kWaitLimitNs))) {
                     fail();
                     ok = false;
@@ -320,7 +320,7 @@ bool prefill_tc_eligible(const Geom &geo)
 {
     // bf16 inputs, a chunk of queries, spans that tile a 32-token warp
     return geo.dtype == REATT_BF16 && geo.C > 1 && (32 % geo.S) == 0 &&
-           int64_t(geo.B) * geo.Hkv * geo.T < (int64_t(1) << 31);
+           int64_t(geo.B) * geo.Hkv * geo.Ts < (int64_t(1) << 31);
 }
 
 static int tc_terms(const Geom &geo) { return geo.g <= 2 ? geo.g : 2; }
@@ -354,7 +354,7 @@ cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, fl
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     CUtensorMap kmap, qmap;
-    if (!make_map(&kmap, kc, uint64_t(geo.B) * geo.Hkv * geo.T, geo.d) ||
+    if (!make_map(&kmap, kc, uint64_t(geo.B) * geo.Hkv * geo.Ts, geo.d) ||
         !make_map(&qmap, terms, uint64_t(geo.B) * geo.Hkv * ta.nterms * ta.cpad, geo.d))
         return cudaErrorInvalidValue;
     int grid = num_sms();

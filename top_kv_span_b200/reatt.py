@@ -20,14 +20,16 @@ F32, BF16 = 0, 1
 
 EXPORTS = ["reatt_status_string", "reatt_num_spans", "reatt_window_max", "reatt_workspace_bytes",
            "reatt_workspace_status", "reatt_score_spans", "reatt_topk", "reatt_gather_rope",
-           "reatt_attend", "reatt_step", "reatt_selftest_bounded_wait", "reatt_step_fixed_scratch"]
+           "reatt_attend", "reatt_step", "reatt_append_kv", "reatt_selftest_bounded_wait",
+           "reatt_step_fixed_scratch"]
 
 
 class reatt_dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("C", ctypes.c_int32), ("G", ctypes.c_int32),
                 ("L", ctypes.c_int32), ("S", ctypes.c_int32), ("k", ctypes.c_int32),
-                ("dtype", ctypes.c_int32), ("T", ctypes.c_int64), ("rope_base", ctypes.c_double)]
+                ("dtype", ctypes.c_int32), ("T", ctypes.c_int64), ("rope_base", ctypes.c_double),
+                ("T_cap", ctypes.c_int64)]
 
 
 class ReattError(RuntimeError):
@@ -55,6 +57,7 @@ lib.reatt_attend.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.reatt_step.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.reatt_step_fixed_scratch.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.reatt_selftest_bounded_wait.argtypes = [_vp, ctypes.c_int64, _vp]
+lib.reatt_append_kv.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp]
 for _name in EXPORTS[1:]:
     getattr(lib, _name).restype = ctypes.c_int
 
@@ -63,13 +66,13 @@ def status_string(code: int) -> str:
     return lib.reatt_status_string(int(code)).decode()
 
 
-def make_dims(B, Hq, Hkv, d, C, T, G, L, S, k, dtype, rope_base) -> reatt_dims:
+def make_dims(B, Hq, Hkv, d, C, T, G, L, S, k, dtype, rope_base, T_cap=0) -> reatt_dims:
     if isinstance(dtype, str):
         dtype = F32 if dtype == "f32" else BF16
     elif isinstance(dtype, torch.dtype):
         dtype = F32 if dtype == torch.float32 else BF16
     return reatt_dims(int(B), int(Hq), int(Hkv), int(d), int(C), int(G), int(L), int(S), int(k),
-                      int(dtype), int(T), float(rope_base))
+                      int(dtype), int(T), float(rope_base), int(T_cap))
 
 
 def dims_of(w, **override) -> reatt_dims:
@@ -167,6 +170,14 @@ def reatt_step(dims, q, k_cache, v_cache, k_cur, v_cur, sel_out, out, ws, stream
                         _ptr(v_cur), _ptr(sel_out), _ptr(out), _ptr(ws), _stream(stream))
     if check:
         _check(rc, "reatt_step")
+    return rc
+
+
+def reatt_append_kv(dims, k_cache, v_cache, k_cur, v_cur, stream=None, check=True):
+    rc = lib.reatt_append_kv(ctypes.byref(dims), _ptr(k_cache), _ptr(v_cache), _ptr(k_cur),
+                             _ptr(v_cur), _stream(stream))
+    if check:
+        _check(rc, "reatt_append_kv")
     return rc
 
 
