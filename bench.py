@@ -38,8 +38,8 @@ PROFILE_SUMMARY = {
 
 
 def step_bytes(w):
-    """Algorithmic bytes one step must move: the middle keys
-    once, the window's K/V rows once, q, the current K/V and the fp32 output."""
+    """Algorithmic bytes one step must move: the middle keys once, the
+    window's K/V rows once, q, the current K/V and the fp32 output."""
     e = w.elem_bytes
     M = max(0, w.T - w.G - w.L)
     scan = w.B * w.Hkv * M * w.d * e

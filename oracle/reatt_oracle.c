@@ -20,7 +20,7 @@
  *          recalled ++ local, then attention.
  *   [HYP]  OpenReview discussion, NIAH comparison settings: global 32,
  *          local 4096, seg_size 32, num_seg 127.
- * Readings where the pages are silent (fixed by the benchmark spec):
+ * Readings taken where the pages are silent:
  *   - a span is S consecutive middle tokens, tiled from the left; the last
  *     span may be short; span score = max over its tokens (and over the
  *     chunk's queries when C > 1);

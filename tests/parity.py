@@ -1,6 +1,6 @@
 """Shared parity checks: CUDA path (through the C ABI) against the CPU oracle.
 
-Acceptance (fixed by the benchmark spec):
+Acceptance bars:
   * selection: the chosen span sets match the oracle's exactly, except swaps
     among spans whose oracle score lies within 1e-3 relative of the oracle's
     k-th score; the number of such swaps is reported;
