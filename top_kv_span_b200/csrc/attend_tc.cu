@@ -83,6 +83,15 @@ __device__ __forceinline__ int64_t row_src_tc(const Geom &geo, const WinMapTc &m
     return (int64_t(1) << 62) | ((bh * geo.C + (p - m.n_loc)) * D);
 }
 
+// 2^x on the special-function unit (ex2.approx.ftz: relative error ~2^-22;
+// 2^-inf = 0), for the softmax numerators.
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo)
 {
     hi = __float2bfloat16_rn(x);
@@ -368,6 +377,8 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
         const uint32_t lane_base = tmem_base + (uint32_t(quad * 32) << 16);
         const bool live = row < nrows;
         const int64_t qpos = live ? qpos0 + (r0 + row) % geo.C : -1;
+        // last key this row sees (window end and causal limit); -1: none
+        const int row_lim = live ? int((kend - 1 < qpos) ? kend - 1 : qpos) : -1;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         uint8_t *ph = smem + Sm::oP, *pl = smem + Sm::oP + Sm::kP;
@@ -393,12 +404,19 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sempty[s]);
+            // keys past this row's limit (window end, causal) are masked;
+            // tiles wholly inside the limit skip the per-key test
             float mx = -INFINITY;
+            const int kb = j * kKeyTile;
+            if (kb + kKeyTile - 1 <= row_lim) {
 #pragma unroll
-            for (int i = 0; i < kKeyTile; ++i) {
-                const int64_t kp = int64_t(j) * kKeyTile + i;
-                if (!(kp < kend && kp <= qpos)) sv[i] = -INFINITY;
-                mx = fmaxf(mx, sv[i]);
+                for (int i = 0; i < kKeyTile; ++i) mx = fmaxf(mx, sv[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < kKeyTile; ++i) {
+                    if (kb + i > row_lim) sv[i] = -INFINITY;
+                    mx = fmaxf(mx, sv[i]);
+                }
             }
             // the P buffer and O are free once P(j-1).V(j-1) has completed
             if (j >= 1) {
@@ -431,15 +449,17 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                 }
             }
             // P = exp2(S - m_ref) as bf16 hi + lo, 128B-swizzled K-major rows
+            const bool any_key = m_ref != -INFINITY;
             float rs = 0.f;
 #pragma unroll
             for (int c = 0; c < kKeyTile / 8; ++c) {
                 uint32_t hw[4], lw[4];
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
-                    float p0 = sv[c * 8 + e] == -INFINITY ? 0.f : exp2f(sv[c * 8 + e] - m_ref);
-                    float p1 = sv[c * 8 + e + 1] == -INFINITY ? 0.f : exp2f(sv[c * 8 + e + 1] - m_ref);
-                    if (!live) p0 = p1 = 0.f;
+                    // masked keys are -inf: ex2 gives 0; a row with no key
+                    // seen yet (m_ref = -inf) has only masked keys
+                    const float p0 = any_key ? ex2_approx(sv[c * 8 + e] - m_ref) : 0.f;
+                    const float p1 = any_key ? ex2_approx(sv[c * 8 + e + 1] - m_ref) : 0.f;
                     rs += p0 + p1;
                     const __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
                     const float2 hf = __bfloat1622float2(hv);
