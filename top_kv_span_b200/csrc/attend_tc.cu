@@ -4,14 +4,15 @@
 // causal attention (ReAttention OpenReview discussion, "Prefilling Phase":
 // flash_attention(query, key_recall, value_recall); research-map summary
 // "Approach": RoPE applied after concatenation, window row p at position p,
-// query c at W-C+c).  To keep fp32-level accuracy with bf16 tensor-core
-// operands every rotated operand is split into bf16 hi + lo:
+// query c at W-C+c).  The rotated operands of the logits are split into bf16
+// hi + lo to keep fp32-level accuracy with bf16 tensor-core operands:
 //   S = Qh.Kh^T + Qh.Kl^T + Ql.Kh^T   (dropped Ql.Kl^T is ~2^-18 relative)
-//   O += Ph.V + Pl.V                  (V is exact: bf16 input)
+// and the probabilities P = exp2(S - m) <= 2^8 meet V in fp16 (11-bit
+// significand, V converted from bf16):  O += P.V.
 //
 // prefill_prep_kernel writes, per KV head, the rotated+scaled query rows
-// (hi/lo), the rotated window keys (hi/lo) and the window values transposed,
-// all bf16, from the un-rotated cache through the selection (the window is
+// (hi/lo), the rotated window keys (hi/lo) and the window values transposed
+// (fp16), from the un-rotated cache through the selection (the window is
 // never materialised in fp32).  attend_prefill_tc_kernel then runs, per
 // 128-row query block:
 //   warp 0   TMA producer: the query block once, then 64-key tiles of K (hi,
@@ -21,11 +22,12 @@
 //   warps 2-5 softmax: one thread per query row reads its S row from TMEM,
 //            masks (causal, window end), keeps a running reference max that
 //            moves (and rescales O in TMEM) only when the row max grows by
-//            more than 2^8, writes P as bf16 hi/lo in the swizzled operand
-//            layout, and finally divides O by the row sum.
+//            more than 2^8, writes P in the swizzled operand layout into one
+//            of two P buffers, and finally divides O by the row sum.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "common.cuh"
@@ -103,7 +105,8 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bflo
 //   kh/kl [BH][Wp][D]  rotated window keys, rows >= W zero
 //   vt    [BH][D][Wp]  window values transposed, columns >= W zero
 struct PrepOut {
-    __nv_bfloat16 *qh, *ql, *kh, *kl, *vt;
+    __nv_bfloat16 *qh, *ql, *kh, *kl;
+    __half *vt;   // fp16: the P.V products take fp16 P
     int Rp, Wp;
 };
 
@@ -154,7 +157,7 @@ prefill_prep_kernel(Geom geo, const uint16_t *__restrict__ q, const uint16_t *__
         __syncthreads();
         for (int x = threadIdx.x; x < D * kPrepRows; x += blockDim.x) {
             const int i = x / kPrepRows, r = x % kPrepRows;
-            po.vt[(bh * D + i) * po.Wp + p0 + r] = __float2bfloat16_rn(vs[r][i]);
+            po.vt[(bh * D + i) * po.Wp + p0 + r] = __float2half_rn(vs[r][i]);
         }
     } else {
         // ---- 64 query rows: rotated at W-C+c, scaled, hi/lo
@@ -221,8 +224,8 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Sm::oBar);
     uint64_t *qfull = bars, *kfull = bars + 1, *kempty = bars + 3, *vfull = bars + 5,
              *vempty = bars + 7, *sfull = bars + 9, *sempty = bars + 11, *pfull = bars + 13,
-             *pvdone = bars + 14, *done = bars + 15;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 16);
+             *pvdone = bars + 15, *done = bars + 17;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -236,9 +239,9 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
             mbar_init(&vempty[s], 1);
             mbar_init(&sfull[s], 1);
             mbar_init(&sempty[s], 4);
+            mbar_init(&pfull[s], 4);     // P buffer s written (one arrival per softmax warp)
+            mbar_init(&pvdone[s], 1);    // P(s).V done: buffer s free again
         }
-        mbar_init(pfull, 4);
-        mbar_init(pvdone, 1);
         mbar_init(done, 1);
         mbar_init_fence();
     }
@@ -314,7 +317,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t id_s = idesc_bf16(kQRows, kKeyTile), id_o = idesc_bf16(kQRows, D);
+            const uint32_t id_s = idesc_bf16(kQRows, kKeyTile), id_o = idesc_f16(kQRows, D);
             bool ok = !aborted() && mbar_wait_bounded(qfull, 0, kWaitLimitNs);
             if (!ok) fail();
             tc_fence_after();
@@ -346,7 +349,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                 }
                 if (j >= 1) {   // O += P(j-1).V(j-1) (hi and lo P)
                     const int jj = j - 1, s = jj & 1;
-                    if (aborted() || !mbar_wait_bounded(pfull, jj & 1, kWaitLimitNs) ||
+                    if (aborted() || !mbar_wait_bounded(&pfull[s], (jj >> 1) & 1, kWaitLimitNs) ||
                         !mbar_wait_bounded(&vfull[s], (jj >> 1) & 1, kWaitLimitNs)) {
                         fail();
                         ok = false;
@@ -357,13 +360,11 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                     const uint8_t *vst = smem + Sm::oV + s * Sm::kV;
 #pragma unroll
                     for (int ks = 0; ks < PS; ++ks) {
-                        const uint64_t ph = sw128_desc(smem + Sm::oP) + uint64_t(ks * 2);
-                        const uint64_t pl = sw128_desc(smem + Sm::oP + Sm::kP) + uint64_t(ks * 2);
+                        const uint64_t pd = sw128_desc(smem + Sm::oP + s * Sm::kP) + uint64_t(ks * 2);
                         const uint64_t vd = sw128_desc(vst) + uint64_t(ks * 2);
-                        tc_mma(d_o, ph, vd, id_o, (jj > 0 || ks > 0) ? 1u : 0u);
-                        tc_mma(d_o, pl, vd, id_o, 1u);
+                        tc_mma(d_o, pd, vd, id_o, (jj > 0 || ks > 0) ? 1u : 0u);
                     }
-                    tc_commit(pvdone);
+                    tc_commit(&pvdone[s]);
                     tc_commit(&vempty[s]);
                 }
             }
@@ -381,7 +382,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
         const int row_lim = live ? int((kend - 1 < qpos) ? kend - 1 : qpos) : -1;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
-        uint8_t *ph = smem + Sm::oP, *pl = smem + Sm::oP + Sm::kP;
+        uint8_t *pbuf = smem + Sm::oP;
         for (int j = 0; j < nt; ++j) {
             const int s = j & 1;
             bool got = !aborted() && mbar_wait_bounded(&sfull[s], (j >> 1) & 1, kWaitLimitNs);
@@ -418,9 +419,9 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                     mx = fmaxf(mx, sv[i]);
                 }
             }
-            // the P buffer and O are free once P(j-1).V(j-1) has completed
-            if (j >= 1) {
-                got = !aborted() && mbar_wait_bounded(pvdone, (j - 1) & 1, kWaitLimitNs);
+            // P buffer j&1 is free once P(j-2).V(j-2) has completed
+            if (j >= 2) {
+                got = !aborted() && mbar_wait_bounded(&pvdone[s], ((j - 2) >> 1) & 1, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, got)) {
                     if (lane == 0) fail();
                     ok = false;
@@ -437,6 +438,16 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                 l *= fac;
             }
             if (j >= 1 && __any_sync(0xffffffffu, move && fac != 1.f)) {
+                // O is quiescent once P(j-1).V(j-1) has completed (P(j).V is
+                // issued only after this tile's P is written)
+                got = !aborted() &&
+                      mbar_wait_bounded(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) fail();
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
                 // rescale this row of O in TMEM (warp-collective accesses)
 #pragma unroll
                 for (int cb = 0; cb < D / 32; ++cb) {
@@ -448,12 +459,14 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                     tmem_st32(ta, o);
                 }
             }
-            // P = exp2(S - m_ref) as bf16 hi + lo, 128B-swizzled K-major rows
+            // P = exp2(S - m_ref) <= 2^8 as fp16 (11-bit significand), 128B-
+            // swizzled K-major rows of buffer j&1
             const bool any_key = m_ref != -INFINITY;
+            uint8_t *pw = pbuf + s * Sm::kP + row * 128;
             float rs = 0.f;
 #pragma unroll
             for (int c = 0; c < kKeyTile / 8; ++c) {
-                uint32_t hw[4], lw[4];
+                uint32_t hw[4];
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     // masked keys are -inf: ex2 gives 0; a row with no key
@@ -461,23 +474,20 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                     const float p0 = any_key ? ex2_approx(sv[c * 8 + e] - m_ref) : 0.f;
                     const float p1 = any_key ? ex2_approx(sv[c * 8 + e + 1] - m_ref) : 0.f;
                     rs += p0 + p1;
-                    const __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
-                    const float2 hf = __bfloat1622float2(hv);
-                    const __nv_bfloat162 lv = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+                    const __half2 hv = __floats2half2_rn(p0, p1);
                     hw[e / 2] = *reinterpret_cast<const uint32_t *>(&hv);
-                    lw[e / 2] = *reinterpret_cast<const uint32_t *>(&lv);
                 }
-                const int phys = (c ^ (row & 7)) * 16;
-                *reinterpret_cast<uint4 *>(ph + row * 128 + phys) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4 *>(pl + row * 128 + phys) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                *reinterpret_cast<uint4 *>(pw + (c ^ (row & 7)) * 16) =
+                    make_uint4(hw[0], hw[1], hw[2], hw[3]);
             }
             l += rs;
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(pfull);
+            if (lane == 0) mbar_arrive(&pfull[s]);
         }
         if (ok && nt > 0) {
-            const bool got = !aborted() && mbar_wait_bounded(pvdone, (nt - 1) & 1, kWaitLimitNs);
+            const bool got = !aborted() &&
+                             mbar_wait_bounded(&pvdone[(nt - 1) & 1], ((nt - 1) >> 1) & 1, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, got)) {
                 if (lane == 0) fail();
             } else {
@@ -588,7 +598,7 @@ cudaError_t launch_attend_prefill_tc(const Geom &geo, const void *q, const void 
     po.ql = reinterpret_cast<__nv_bfloat16 *>(base + pp.q_bytes);
     po.kh = reinterpret_cast<__nv_bfloat16 *>(base + 2 * pp.q_bytes);
     po.kl = reinterpret_cast<__nv_bfloat16 *>(base + 2 * pp.q_bytes + pp.k_bytes);
-    po.vt = reinterpret_cast<__nv_bfloat16 *>(base + 2 * pp.q_bytes + 2 * pp.k_bytes);
+    po.vt = reinterpret_cast<__half *>(base + 2 * pp.q_bytes + 2 * pp.k_bytes);
     po.Rp = pp.Rp;
     po.Wp = pp.Wp;
     const unsigned BH = unsigned(geo.B * geo.Hkv);

@@ -172,6 +172,11 @@ __device__ __forceinline__ uint64_t sw128_mn_desc(const void *p, uint32_t lbo)
     d |= 2ull << 61;                                   // 128-byte swizzle
     return d;
 }
+// Instruction descriptor, kind::f16: fp32 D, fp16 A and B, both K-major, M x N.
+constexpr uint32_t idesc_f16(int M, int N)
+{
+    return (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
 // Instruction descriptor as idesc_bf16 with A read MN-major (transposed).
 constexpr uint32_t idesc_bf16_amn(int M, int N) { return idesc_bf16(M, N) | (1u << 15); }
 
