@@ -143,6 +143,14 @@ def aggregate(world, step_b, steps, total_ms, e2e_ms, scan_ms, reduce_max=None):
             "e2e_value": world * step_b * steps / (e2e_ms * 1e-3) / 1e9}
 
 
+def config_of(w, world):
+    """The workload named by its sizes (both arms print the same dict)."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "C": w.C,
+            "T": w.T, "G": w.G, "L": w.L, "S": w.S, "k": w.k, "rope_base": w.rope_base,
+            "parallelism": f"replicas x{world}",
+            "l2": "flushed before every step (512 MiB read); flush outside the step events"}
+
+
 def dist_us(ms_list):
     """Median, p10 and p90 (µs) of a list of per-step times in ms."""
     v = sorted(ms_list)
@@ -344,10 +352,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": w.dtype,
         "data": "synthetic (seeded caches, per-channel sigma, planted needles)",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "C": w.C,
-                   "T": w.T, "G": w.G, "L": w.L, "S": w.S, "k": w.k, "rope_base": w.rope_base,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "flushed before every step (512 MiB read); flush outside the step events"},
+        "config": config_of(w, world),
         "roofline": roofline(w, scan_b, scan_ms),
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms / args.steps * 1e3, 2)},
@@ -433,7 +438,7 @@ def run_reference(args):
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "parallelism": "host cores (OpenMP)"},
+        "config": config_of(w, 1),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.max_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
