@@ -148,3 +148,41 @@ def test_topk_negative_and_infinite_scores(R):
     torch.cuda.synchronize()
     order = np.lexsort((np.arange(NS), -sc.astype(np.float64)))
     assert sel.cpu().numpy()[0, 0].tolist() == sorted(order[:w.k].tolist())
+
+
+@pytest.mark.parametrize("dist", ["normal", "ties", "narrow", "equal", "wide"])
+def test_topk_sizes_and_value_spreads(R, dist):
+    """The selection against its definition (score descending, ties to the lower
+    span id, the first k_eff ids, ascending) over one-slice and multi-slice span
+    counts, k around and above the span count, and several heads at once."""
+    rng = np.random.default_rng(["normal", "ties", "narrow", "equal", "wide"].index(dist) + 40)
+    for NS, k in [(1, 1), (7, 3), (7, 9), (100, 64), (3967, 64), (4096, 64), (4097, 64),
+                  (5000, 1), (9000, 200), (20000, 64), (2048, 2048)]:
+        w = LLAMA.replace(B=2, Hq=4, Hkv=2, d=64, T=32 + 4096 + 32 * NS, G=32, L=4096, S=32, k=k)
+        d = R.dims_of(w)
+        assert R.reatt_num_spans(d) == NS
+        shape = (w.B, w.Hkv, NS)
+        if dist == "normal":
+            sc = rng.standard_normal(shape)
+        elif dist == "ties":
+            sc = rng.integers(0, 5, shape)
+        elif dist == "narrow":
+            sc = 100.0 + 1e-4 * rng.standard_normal(shape)
+        elif dist == "equal":
+            sc = np.full(shape, 3.5)
+        else:
+            sc = rng.standard_normal(shape) * 10.0 ** rng.integers(-30, 30, shape)
+        sc = sc.astype(np.float32)
+        scores = torch.tensor(sc).cuda()
+        sel = torch.full((w.B, w.Hkv, k), 12345, dtype=torch.int32, device="cuda")
+        ws = torch.empty(R.reatt_workspace_bytes(d), dtype=torch.uint8, device="cuda")
+        R.reatt_topk(d, scores, sel, ws)
+        torch.cuda.synchronize()
+        got = sel.cpu().numpy()
+        keff = min(k, NS)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                s = sc[b, h].astype(np.float64)
+                order = np.lexsort((np.arange(NS), -s))
+                want = sorted(order[:keff].tolist()) + [-1] * (k - keff)
+                assert got[b, h].tolist() == want, (dist, NS, k, b, h)
