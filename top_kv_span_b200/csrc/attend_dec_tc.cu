@@ -15,7 +15,8 @@
 //               columns, 128B-swizzled, each inside one run of the window (the
 //               global part, a chosen span, the local part, the current tokens)
 //               and one 32-row quarter of the tile, which has its own barrier;
-//               V lands directly in the MN-major operand layout
+//               lane q issues quarter q, so the four quarters' loads go out
+//               together; V lands directly in the MN-major operand layout
 //   warp 1      TMEM allocation; one thread issues S(j) and then P(j-1).V(j-1)
 //   warps 2-9   rotate the raw keys of each quarter as it lands (RoPE with
 //               the step's cos/sin table) and split them into the hi/lo
@@ -252,15 +253,14 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                 if (lane == 0) fail();
                 break;
             }
-            if (lane == 0) {
+            if (lane < 4) {
+                // lane q issues quarter q (rows [32q, 32q + 32) of the tile):
+                // its expected bytes, then its boxes
+                const int q = lane;
                 int p0, n;
                 tile_at(j, p0, n);
-                // every run of the window starts at a multiple of 8 rows, so
-                // the boxes cover roundup(n, 8) rows
-                // bytes per 32-row quarter: K and V rows (both halves), plus
-                // the V pad box of an odd last group; one arrival each
                 const int ng = (n + 7) / 8;
-                for (int q = 0; q < 4; ++q) {
+                {
                     int rows = 8 * ng - kDtQuarter * q;
                     rows = rows < 0 ? 0 : (rows > kDtQuarter ? kDtQuarter : rows);
                     uint32_t bytes = uint32_t(rows) * 512u;
@@ -271,8 +271,9 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                         mbar_arrive(&tq[4 * s + q]);
                 }
                 uint8_t *kst = smem + Sm::oRaw + s * kDtTile, *vst = smem + Sm::oV + s * kDtTile;
-                for (int r = 0; r < n;) {
-                    // the run holding window row p0 + r and that row's source
+                const int r_end = kDtQuarter * q + kDtQuarter < n ? kDtQuarter * q + kDtQuarter : n;
+                uint64_t *bar = &tq[4 * s + q];
+                for (int r = kDtQuarter * q; r < r_end;) {
                     const int p = p0 + r;
                     int run_end;
                     bool cur = false;
@@ -281,7 +282,7 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                         run_end = g_end;
                         y = bh * geo.Ts + p;
                     } else if (p - g_end < nsel) {
-                        const int q = p - g_end, jj = q / geo.S, off = q - jj * geo.S;
+                        const int qq = p - g_end, jj = qq / geo.S, off = qq - jj * geo.S;
                         int sp = sel_cached ? sel_s[jj - j0] : sel_bh[jj];
                         sp = sp < 0 ? 0 : (sp >= int(geo.NS) ? int(geo.NS) - 1 : sp);
                         run_end = g_end + (jj + 1) * geo.S;
@@ -294,24 +295,19 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                         cur = true;
                         y = bh * geo.C + (p - g_end - nsel - nloc);
                     }
-                    int len = (run_end < p0 + n ? run_end : p0 + n) - p;
+                    int len = (run_end < p0 + r_end ? run_end : p0 + r_end) - p;
                     while (len > 0) {
-                        // 32-row boxes start on a quarter, so none crosses one
                         const int hs = (!cur && len >= 32 && (r & 31) == 0) ? 0 : 1;
                         const CUtensorMap *km = cur ? &maps.kq : &maps.k[hs];
                         const CUtensorMap *vm = cur ? &maps.vq : &maps.v[hs];
-                        uint64_t *bar = &tq[4 * s + r / kDtQuarter];
                         tma_load_2d(kst + r * 128, km, 0, int(y), bar);
                         tma_load_2d(kst + kDtHalf + r * 128, km, 64, int(y), bar);
                         tma_load_2d(vst + r * 128, vm, 0, int(y), bar);
                         tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), bar);
                         r += dt_box_rows(hs);
                         if (r >= n && (r & 8)) {
-                            // odd number of 8-row groups: one more box of the
-                            // same rows fills the tile's last 16-key step
-                            uint64_t *pbar = &tq[4 * s + r / kDtQuarter];
-                            tma_load_2d(vst + r * 128, vm, 0, int(y), pbar);
-                            tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), pbar);
+                            tma_load_2d(vst + r * 128, vm, 0, int(y), bar);
+                            tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), bar);
                         }
                         y += dt_box_rows(hs);
                         len -= dt_box_rows(hs);
