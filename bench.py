@@ -381,26 +381,41 @@ def oracle_sample(w, x, heads):
     return {n: wl.to_oracle(t) for n, t in sub.items()}, w.replace(B=1, Hkv=heads, Hq=heads * g)
 
 
-def cpu_baseline(w, x, seconds=15.0, heads=None):
+def cpu_baseline(w, x, seconds=15.0, heads=None, single_seconds=5.0):
     """The oracle as it stands, on this host's cores, over a bounded sample of
-    the workload (the first KV head(s) of sequence 0), repeated for ~seconds."""
+    the workload (the first KV head(s) of sequence 0), repeated for ~seconds;
+    then the same sample on one core for ~single_seconds."""
     import oracle
     heads = heads or 1
     xs, ws = oracle_sample(w, x, heads)
     _, sb = step_bytes(ws)
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        oracle.step(**xs, G=ws.G, L=ws.L, S=ws.S, k=ws.k, rope_base=ws.rope_base,
-                    want_scores=False)
-        n += 1
-        if time.perf_counter() - t0 > seconds:
-            break
-    dt = (time.perf_counter() - t0) / n
-    return {"value": round(sb / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.max_threads(),
-            "kind": "oracle", "sample": f"{w.name}: sequence 0, {heads} of {w.Hkv} KV heads "
-                                        f"({heads * (w.Hq // w.Hkv)} query heads), {n} oracle steps",
-            "sec_per_sample_step": round(dt, 4)}
+
+    def timed(limit):
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            oracle.step(**xs, G=ws.G, L=ws.L, S=ws.S, k=ws.k, rope_base=ws.rope_base,
+                        want_scores=False)
+            n += 1
+            if time.perf_counter() - t0 > limit:
+                break
+        return (time.perf_counter() - t0) / n, n
+
+    cores = oracle.max_threads()
+    dt, n = timed(seconds)
+    out = {"value": round(sb / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
+           "kind": "oracle", "sample": f"{w.name}: sequence 0, {heads} of {w.Hkv} KV heads "
+                                       f"({heads * (w.Hq // w.Hkv)} query heads), {n} oracle steps",
+           "sec_per_sample_step": round(dt, 4)}
+    if single_seconds > 0:
+        oracle.set_threads(1)
+        try:
+            dt1, n1 = timed(single_seconds)
+        finally:
+            oracle.set_threads(cores)
+        out["single_thread"] = {"value": round(sb / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                                "sec_per_sample_step": round(dt1, 4), "steps": n1}
+    return out
 
 
 def run_reference(args):
