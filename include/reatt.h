@@ -24,7 +24,9 @@
  *   M = max(0, T-G-L), NS = ceil(M/S) spans tiled from the left (the last one
  *   may be short), k_eff = min(k, NS),
  *   W = min(G,T) + (rows of the chosen spans) + (T - max(G, T-L) if T > G) + C,
- *   Wmax = G + k*S + L + C  (an upper bound on W).
+ *   Wmax = G + k*S + L + C  (an upper bound on W; at most 2^24, since window
+ *   positions enter the RoPE angle as exact fp32 integers; larger windows are
+ *   REATT_EUNSUPPORTED).
  *
  * Conventions for every entry point
  *   - Layouts are contiguous row-major:
@@ -213,9 +215,11 @@ REATT_API int reatt_selftest_bounded_wait(void *ws, int64_t limit_ns, reatt_stre
  * bf16 prefill chunk over 256K tokens needs 92.7 MiB (its tensor-core
  * attention operands) and is rejected.
  *   - Allocates nothing: no cudaMalloc/cudaFree or allocating library call.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, which also loads the library's device globals
- *     there); make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress; nothing is cached, so the call stays valid after
+ *     a cudaDeviceReset).  The first call on a device also loads the
+ *     library's device globals there; make that first call before any stream
+ *     capture.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents; what must start at zero is cleared inside each call.  Calls
  *     that overlap on the GPU race: order them on one stream.

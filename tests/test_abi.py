@@ -98,6 +98,8 @@ def test_workspace_grows_with_spans(R):
     (dict(rope_base=0.0), 1), (dict(rope_base=float("inf")), 1), (dict(rope_base=float("nan")), 1),
     (dict(d=96), 2), (dict(d=256), 2), (dict(dtype=7), 2), (dict(k=70000), 2),
     (dict(T=1 << 31), 2),
+    # window positions past 2^24 are not exact fp32 integers in the RoPE angle
+    (dict(S=1 << 14, k=1 << 10), 2),
 ])
 def test_bad_dims_rejected_everywhere(R, bad, code):
     d = dims(R, **bad)
@@ -147,3 +149,13 @@ def test_null_and_misaligned_pointers(R):
     assert R.reatt_attend(d, A, A, A, A, M, A, stream=0, check=False) == 1
     assert R.reatt_step(d, A, A, A, A, A, M, A, A, stream=0, check=False) == 1
     assert R.reatt_step(d, A, A, A, A, A, None, A, M, stream=0, check=False) == 1
+
+
+def test_window_limit_is_two_to_the_24(R):
+    # Wmax = G + k*S + L + C: exactly 2^24 is accepted, one more is not
+    v = ctypes.c_int64()
+    ok = dims(R, G=0, L=0, C=1, S=(1 << 24) - 1, k=1)
+    assert R.lib.reatt_window_max(ctypes.byref(ok), ctypes.byref(v)) == R.OK
+    assert v.value == 1 << 24
+    bad = dims(R, G=0, L=0, C=2, S=(1 << 24) - 1, k=1)
+    assert R.lib.reatt_window_max(ctypes.byref(bad), ctypes.byref(v)) == R.EUNSUPPORTED

@@ -12,6 +12,7 @@ namespace {
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+constexpr int64_t kMaxWindow = int64_t(1) << 24;   // Wmax limit (exact fp32 positions)
 
 int make_geom(const reatt_dims *d, Geom *g)
 {
@@ -27,7 +28,9 @@ int make_geom(const reatt_dims *d, Geom *g)
     if (d->T >= (int64_t(1) << 31)) return REATT_EUNSUPPORTED;
     if (d->T_cap != 0 && (d->T_cap < d->T || d->T_cap >= (int64_t(1) << 31))) return REATT_EINVAL;
     const double wmax = double(d->G) + double(d->k) * d->S + d->L + d->C;
-    if (wmax >= 2147483647.0) return REATT_EUNSUPPORTED;
+    // RoPE angles are formed from the window position in fp32 (rope_cs), which
+    // holds every integer position exactly only below 2^24.
+    if (wmax > double(kMaxWindow)) return REATT_EUNSUPPORTED;
     // element counts of the largest buffers must fit comfortably in int64
     const double cache = double(d->B) * d->Hkv * double(d->T_cap ? d->T_cap : d->T) * d->d;
     const double win = double(d->B) * d->Hkv * wmax * d->d;

@@ -5,8 +5,6 @@
 // workspace is a file-scope __device__ array of fixed size that lives as long
 // as the library is loaded (each GPU that loads the library holds it until the
 // process exits).
-#include <mutex>
-
 #include <cuda_runtime.h>
 
 #include "reatt.h"
@@ -19,23 +17,16 @@ constexpr size_t kFixedScratchBytes = size_t(16) << 20;   // 16 MiB
 // its device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void *g_ptr[kMaxDevices];
-
-// Device address of the scratch on the current device; resolved once per
-// device (the first call loads the module's globals on that device).
+// Device address of the scratch on the current device, looked up on every
+// call (a lookup, no synchronisation).  Nothing is cached: after a
+// cudaDeviceReset the library's globals are loaded again into the new context,
+// possibly at another address, and a cached pointer would be stale.  The first
+// lookup on a device loads the module's globals there.
 int scratch_on_current_device(void **out)
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return REATT_ECUDA;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_fixed_scratch) != cudaSuccess || !p) return REATT_ECUDA;
-        g_ptr[dev] = p;
-    }
-    *out = g_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fixed_scratch) != cudaSuccess || !p) return REATT_ECUDA;
+    *out = p;
     return REATT_OK;
 }
 

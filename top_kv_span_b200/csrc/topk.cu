@@ -4,10 +4,15 @@
 // emitted in ascending span order so the window keeps cache order.
 //
 // Scores are mapped to order-preserving uint32 codes.  A block radix select
-// (4 passes of 8 bits, shared-memory histogram, one warp scans the bins) finds
-// the code tau of the k-th largest and how many codes equal to tau are taken;
-// a stable block compaction in index order then writes the chosen ids, which
-// are therefore already ascending -- no sort is needed.
+// finds the code tau of the k-th largest and how many codes equal to tau are
+// taken.  The path every slice and merge of up to 8192 codes takes keeps the
+// codes in registers, skips the high bits that the block's largest and
+// smallest code share, resolves the rest with 11-bit digits (2048-bin
+// shared-memory histogram) and, once at most 32 codes share the digit prefix,
+// lets one warp rank them directly.  Larger candidate sets fall back to a
+// generic select of 4 passes of 8 bits read from memory.  A stable block
+// compaction in index order then writes the chosen ids, which are therefore
+// already ascending -- no sort is needed.
 // NS <= kSlice: one CTA per head.  Larger NS: slice CTAs (kSlice scores each)
 // emit their own top-k candidates in index order, and one merge CTA per head
 // runs the same select on the candidates.  The global top-k under the total
