@@ -2,18 +2,28 @@
 
 One step = one pass of the whole hot path over one batch: span scoring of the
 middle of the pre-RoPE cache, top-k span selection, and attention over the
-RoPE'd window (reatt_step through the C ABI).  Default workload: the
+RoPE'd window (reatt_step through the C ABI).  Headline workload: the
 LLaMA3-8B-shaped 128K-context bf16 decode (B=1, 32/8 heads, d=128, G=32,
 L=4096, S=32, k=64).  Inputs are seeded synthetic caches resident in HBM;
 L2 is flushed (a 512 MiB read) before every timed step and the flush is
 outside each step's CUDA-event interval.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference] [--extra NAMES] [--loops NAMES]
 
-Multi-GPU (torchrun, one process per GPU): every rank runs its own replica
-sequence(s) -- the path has no cross-sequence exchange -- and rank 0 prints
-the aggregate over ranks with the max per-rank time ("scaling": "weak").
-`--impl reference` times the CPU oracle on the host cores instead.
+At N=1 the same line also carries `per_workload` (the other workloads: the
+tiny fp32 decode, the 1M x 4 and 4M decodes, the 2048-query prefill chunk),
+each with its own timings, roofline and a parity sample, and `decode_loop`
+(a graph-replayed decoding loop with its appends).  Parity comes from the
+CPU leg, which runs the oracle on a bounded sample (KV head 0 of sequence 0)
+and compares the GPU's selection (swap count) and outputs (max-abs) on it.
+
+Multi-GPU: `--gpus N` starts N ranks of this script under
+torch.distributed.run (one process per GPU) unless a launcher already did;
+every rank runs its own replica sequence(s) -- the path has no
+cross-sequence exchange -- and rank 0 prints the aggregate over ranks with
+the max per-rank time ("scaling": "weak").  `--impl reference` times the CPU
+oracle on the host cores instead.
 """
 from __future__ import annotations
 
@@ -195,100 +205,161 @@ def roofline(w, scan_b, scan_ms):
             "bytes_per_launch": scan_b}
 
 
-def dist_setup(n_gpus):
+def dist_setup(cpu=False):
+    """Rank, world and local rank from the launcher's environment; a process
+    group over NCCL (one GPU per rank) or, for the CPU launch check, gloo."""
+    import datetime
+
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if cpu:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        else:
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
     return world, rank, local
 
 
-def run_ours(args):
+def host_cores():
+    """Cores this process may run on (a launcher may have set OMP_NUM_THREADS=1)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def free_port():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def relaunch(n, argv):
+    """`--gpus N` without a launcher around us: start N ranks of this script
+    under torch.distributed.run (one process per GPU, rendezvous on
+    127.0.0.1) and return the launcher's exit code."""
+    import subprocess
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def make_reduce_max(world, dev=None):
     import torch
     import torch.distributed as dist
 
-    world, rank, local = dist_setup(args.gpus)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
+    def reduce_max(vals):
+        t = torch.tensor(vals, dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return [float(v) for v in t.tolist()]
+    return reduce_max if world > 1 else None
+
+
+def run_launch_check(args):
+    """The multi-rank plumbing without a GPU (gloo): every rank reports its
+    own replica times, rank 0 prints the job line (max time over ranks,
+    bytes of every rank)."""
+    import torch.distributed as dist
+    world, rank, _ = dist_setup(cpu=True)
+    total, e2e, scan = 10.0 + rank, 12.0 + 3 * rank, 5.0 - 0.5 * rank
+    agg = aggregate(world, 1_000_000, args.steps, total, e2e, scan, make_reduce_max(world))
+    if rank == 0:
+        print(json.dumps({"launch_check": True, "n_gpus": world, "steps": args.steps,
+                          "total_ms": agg["total_ms"], "e2e_ms": agg["e2e_ms"],
+                          "scan_ms": agg["scan_ms"], "value": agg["value"]}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+class Timer:
+    """Per-step device times with CUDA events on the launching stream, L2
+    flushed (a 512 MiB read) before each step outside the events."""
+
+    def __init__(self, dev, stream):
+        import torch
+        self.torch, self.dev, self.stream = torch, dev, stream
+        self.flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.flush_buf.fill_(1)
+
+    def flush(self):
+        self.flush_buf.sum(dtype=self.torch.int32)   # a full read: L2 ends up holding unrelated lines
+
+    def run(self, fn, steps, warmup=0, flush=True):
+        torch = self.torch
+        for _ in range(warmup):
+            if flush:
+                self.flush()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            if flush:
+                self.flush()
+            ev[i][0].record(self.stream)
+            fn(i)
+            ev[i][1].record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        return [a.elapsed_time(b) for a, b in ev]
+
+
+def launches_per_step(step):
+    """Our kernels in one step, counted once with the profiler (outside timing)."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    step()
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        step()
+        torch.cuda.synchronize()
+    return sum(1 for e in prof.events() if e.device_type.name == "CUDA" and "reatt" in e.name)
+
+
+def measure(w, args, dev, timer, world=1, rank=0, cpu_leg_seconds=0.0, single_seconds=0.0):
+    """One workload: step, scan alone and end-to-end timings, roofline of the
+    scan, and (rank 0) the CPU leg: the oracle on a bounded sample, which
+    also yields the parity of that sample (selection swaps, max-abs)."""
+    import torch
     from top_kv_span_b200 import reatt as R
     from top_kv_span_b200 import workloads as wl
 
-    w = wl.WORKLOADS[args.workload]
-    # weak scaling: rank r runs its own sequences (seed offset by rank)
-    w = w.replace(seed=w.seed + 1000 * rank)
     x = wl.make_inputs(w, dev)
     d = R.dims_of(w)
     buf = R.alloc_outputs(d, device=dev)
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    flush.fill_(1)
 
-    def do_flush():
-        flush.sum(dtype=torch.int32)   # a full read: L2 ends up holding unrelated clean lines
-
-    def step():
+    def step(i=0):
         R.reatt_step(d, x["q"], x["k_cache"], x["v_cache"], x["k_cur"], x["v_cur"], buf["sel"],
                      buf["out"], buf["ws"], stream)
 
-    def scan_only():
+    def scan_only(i=0):
         R.reatt_score_spans(d, x["q"], x["k_cache"], buf["span_scores"], buf["ws"], stream)
 
-    # our kernels per step, counted once with the profiler (outside timing)
-    from torch.profiler import ProfilerActivity, profile
-    step()
-    torch.cuda.synchronize(dev)
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        step()
-        torch.cuda.synchronize(dev)
-    per_step = sum(1 for e in prof.events()
-                   if e.device_type.name == "CUDA" and "reatt" in e.name)
-
-    for _ in range(args.warmup):
-        do_flush()
-        step()
-    torch.cuda.synchronize(dev)
-    assert R.reatt_workspace_status(buf["ws"], stream) == R.OK
-
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    per_step = launches_per_step(step)
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(dev) as clk:
-        for i in range(args.steps):
-            do_flush()
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize(dev)
+        step_ms = timer.run(step, args.steps, warmup=args.warmup)
     if world > 1:
         dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-
-    # dominant kernel (span scan) timed alone, same launch configuration
-    for _ in range(3):
-        do_flush()
-        scan_only()
-    sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.steps):
-        do_flush()
-        sev[i][0].record(stream)
-        scan_only()
-        sev[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    scan_list = [a.elapsed_time(b) for a, b in sev]
-    scan_ms = statistics.mean(scan_list)
+    assert R.reatt_workspace_status(buf["ws"], stream) == R.OK
+    gpu_sel = buf["sel"].cpu().numpy()
+    gpu_out = buf["out"].cpu().numpy()
+    scan_list = timer.run(scan_only, args.steps, warmup=3)
 
     # end to end through the C ABI with host buffers: per step the new
-    # token's q / k / v go host->device from pinned memory and the output
+    # tokens' q / k / v go host->device from pinned memory and the output
     # comes back; the KV cache is device-resident state, as in decoding.  The
     # three inputs sit back to back in one pinned staging buffer (and one
     # device buffer), so a step needs one host->device copy.
@@ -304,66 +375,192 @@ def run_ours(args):
         n = t.numel() * t.element_size()
         hbuf[o:o + n].copy_(t.cpu().contiguous().view(torch.uint8).reshape(-1))
         views.append(dbuf[o:o + n].view(t.dtype).view(t.shape))
+    host_x = {n: x[n] for n in ("q", "k_cur", "v_cur")}
     x["q"], x["k_cur"], x["v_cur"] = views
     hout = torch.empty(buf["out"].shape, dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in parts)
     d2h = hout.numel() * 4
-    for _ in range(3):
-        dbuf.copy_(hbuf, non_blocking=True)
-        step()
-    torch.cuda.synchronize(dev)
-    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.steps):
-        do_flush()
-        eev[i][0].record(stream)
+
+    def e2e_step(i=0):
         dbuf.copy_(hbuf, non_blocking=True)
         step()
         hout.copy_(buf["out"], non_blocking=True)
-        eev[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = sum(a.elapsed_time(b) for a, b in eev)
 
-    def reduce_max(vals):
-        t = torch.tensor(vals, dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return [float(v) for v in t.tolist()]
+    e2e_list = timer.run(e2e_step, args.steps, warmup=3)
+    x.update(host_x)
 
+    res = {"w": w, "x": x, "per_step": per_step, "clk": clk.summary(),
+           "step_ms": step_ms, "scan_ms": scan_list, "e2e_ms": e2e_list,
+           "h2d": h2d, "d2h": d2h}
+    if rank == 0 and (cpu_leg_seconds >= 0):
+        res["cpu"] = cpu_leg(w, x, gpu_sel, gpu_out, seconds=cpu_leg_seconds,
+                             single_seconds=single_seconds)
+    del buf
+    return res
+
+
+def summarise(res, world=1, steps=None, reduce_max=None):
+    """JSON fields of one measured workload (times: max over ranks)."""
+    w = res["w"]
+    steps = steps or len(res["step_ms"])
     scan_b, step_b = step_bytes(w)
-    agg = aggregate(world, step_b, args.steps, total_ms, e2e_ms, scan_ms,
-                    reduce_max if world > 1 else None)
-    total_ms, e2e_ms, scan_ms = agg["total_ms"], agg["e2e_ms"], agg["scan_ms"]
-    ms_per_step = total_ms / args.steps
-    value, e2e_value = agg["value"], agg["e2e_value"]
-    achieved = scan_b / (scan_ms * 1e-3) / 1e9
-    result = {
-        "metric": METRIC,
-        "value": round(value, 1),
+    agg = aggregate(world, step_b, steps, sum(res["step_ms"]), sum(res["e2e_ms"]),
+                    statistics.mean(res["scan_ms"]), reduce_max)
+    ms_per_step = agg["total_ms"] / steps
+    out = {
+        "value": round(agg["value"], 1),
         "unit": "GB/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 5),
         "step_us": round(ms_per_step * 1e3, 2),
-        "scan_us": round(scan_ms * 1e3, 2),
-        "scan_gbs": round(achieved, 1),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
+        "scan_us": round(agg["scan_ms"] * 1e3, 2),
+        "scan_gbs": round(scan_b / (agg["scan_ms"] * 1e-3) / 1e9, 1),
         "dtype": w.dtype,
-        "data": "synthetic (seeded caches, per-channel sigma, planted needles)",
         "config": config_of(w, world),
-        "roofline": roofline(w, scan_b, scan_ms),
-        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "us_per_step": round(e2e_ms / args.steps * 1e3, 2)},
-        "gpu_launches": per_step * args.steps,
-        "clocks": clk.summary(),
+        "roofline": roofline(w, scan_b, agg["scan_ms"]),
+        "step_roofline": step_roofline(w, ms_per_step),
+        "e2e": {"value": round(agg["e2e_value"], 1), "unit": "GB/s",
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+                "us_per_step": round(agg["e2e_ms"] / steps * 1e3, 2)},
+        "gpu_launches": res["per_step"] * steps,
+        "clocks": res["clk"],
         # this rank's distribution over the timed steps (µs): median, p10, p90
-        "step_dist_us": dist_us(step_ms),
-        "scan_dist_us": dist_us(scan_list),
+        "step_dist_us": dist_us(res["step_ms"]),
+        "scan_dist_us": dist_us(res["scan_ms"]),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, x, seconds=args.cpu_seconds)
+    if "cpu" in res:
+        cpu = dict(res["cpu"])
+        out["parity"] = cpu.pop("parity")
+        if cpu.get("value") is not None:
+            out["cpu_baseline"] = cpu
+    return out
+
+
+def step_roofline(w, ms_per_step):
+    """The whole step against its bytes-over-HBM time (decode) or its
+    flops-over-tensor time (bf16 prefill chunk)."""
+    hbm, tflops, kind = peaks()
+    _, step_b = step_bytes(w)
+    if w.C > 1 and w.dtype == "bf16" and 32 % w.S == 0:
+        fl = scan_flops(w) + attn_flops(w)
+        t = fl / (tflops * 1e12)
+        return {"bound": "tensor", "flops": fl, "roofline_us": round(t * 1e6, 2),
+                "frac": round(t / (ms_per_step * 1e-3), 4), "peak_kind": kind}
+    t = step_b / (hbm * 1e9)
+    return {"bound": "hbm", "bytes": step_b, "roofline_us": round(t * 1e6, 2),
+            "frac": round(t / (ms_per_step * 1e-3), 4), "peak_kind": kind}
+
+
+def attn_flops(w):
+    """Algorithmic flops of the window attention of a chunk: q.k and p.v over
+    the causal window, 4*d per (query row, visible key)."""
+    win_cached = min(w.G, w.T) + min(w.k * w.S, max(0, w.T - w.G - w.L)) + \
+        (w.T - max(w.G, w.T - w.L) if w.T > w.G else 0)
+    visible = w.C * win_cached + w.C * (w.C + 1) // 2
+    return 4 * w.B * w.Hq * visible * w.d
+
+
+def decode_loop(w, dev, timer, n_steps=16, reps=10):
+    """NEXT step of a decoding loop, as a caller runs it: n_steps decode
+    steps, each followed by the append of its token's K/V, captured once in
+    a CUDA graph on caches with room to grow (T_cap = T + n_steps) and
+    replayed.  Returns µs per step for the replayed graph and for the same
+    loop launched eagerly (L2 flushed before each loop, not between its
+    steps)."""
+    import torch
+    from top_kv_span_b200 import reatt as R
+    from top_kv_span_b200 import workloads as wl
+
+    x = wl.make_inputs(w, dev)
+    cap = w.T + n_steps
+    shape = (w.B, w.Hkv, cap, w.d)
+    kc = torch.zeros(shape, dtype=w.torch_dtype, device=dev)
+    vc = torch.zeros(shape, dtype=w.torch_dtype, device=dev)
+    kc[:, :, :w.T] = x["k_cache"]
+    vc[:, :, :w.T] = x["v_cache"]
+    del x
+    gen = torch.Generator(device=dev).manual_seed(w.seed + 77)
+    rnd = lambda shp: torch.randn(shp, generator=gen, device=dev).to(w.torch_dtype)
+    qs = [rnd((w.B, w.Hq, 1, w.d)) for _ in range(n_steps)]
+    kn = [rnd((w.B, w.Hkv, 1, w.d)) for _ in range(n_steps)]
+    vn = [rnd((w.B, w.Hkv, 1, w.d)) for _ in range(n_steps)]
+    dims = [R.dims_of(w, T=w.T + i, T_cap=cap) for i in range(n_steps)]
+    ws = torch.zeros(max(R.reatt_workspace_bytes(dd) for dd in dims), dtype=torch.uint8,
+                     device=dev)
+    outs = [torch.empty((w.B, w.Hq, 1, w.d), dtype=torch.float32, device=dev)
+            for _ in range(n_steps)]
+    sels = [torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev)
+            for _ in range(n_steps)]
+    st = torch.cuda.Stream(dev)
+
+    def loop(stream):
+        for i in range(n_steps):
+            R.reatt_step(dims[i], qs[i], kc, vc, kn[i], vn[i], sels[i], outs[i], ws,
+                         stream=stream)
+            R.reatt_append_kv(dims[i], kc, vc, kn[i], vn[i], stream=stream)
+
+    with torch.cuda.stream(st):
+        loop(st)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=st):
+            loop(st)
+        t = Timer(dev, st)
+        g_ms = t.run(lambda i=0: graph.replay(), reps, warmup=3)
+        e_ms = t.run(lambda i=0: loop(st), reps, warmup=3)
+    assert R.reatt_workspace_status(ws, st) == R.OK
+    del graph
+    return {"steps_per_loop": n_steps, "T_first": w.T,
+            "graph_us_per_step": round(statistics.median(g_ms) * 1e3 / n_steps, 2),
+            "eager_us_per_step": round(statistics.median(e_ms) * 1e3 / n_steps, 2),
+            "note": "median over replays; one L2 flush before each loop of steps"}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_setup()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {world} ranks")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from top_kv_span_b200 import workloads as wl
+
+    stream = torch.cuda.current_stream(dev)
+    timer = Timer(dev, stream)
+    w = wl.WORKLOADS[args.workload]
+    # weak scaling: rank r runs its own sequences (seed offset by rank)
+    w = w.replace(seed=w.seed + 1000 * rank)
+    head = measure(w, args, dev, timer, world, rank,
+                   cpu_leg_seconds=-1 if (world > 1 or args.no_cpu_baseline) else args.cpu_seconds,
+                   single_seconds=args.cpu_single_seconds)
+    line = summarise(head, world, args.steps, make_reduce_max(world, dev))
+    result = {"metric": METRIC, "value": line.pop("value"), "unit": line.pop("unit"),
+              "n_gpus": world, "steps": args.steps, "warmup": args.warmup}
+    result.update({k: line[k] for k in ("ms_per_step", "step_us", "scan_us", "scan_gbs")})
+    result.update({"higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                   "dtype": line["dtype"],
+                   "data": "synthetic (seeded caches, per-channel sigma, planted needles)"})
+    for k in ("config", "roofline", "step_roofline", "e2e", "gpu_launches", "clocks",
+              "step_dist_us", "scan_dist_us", "parity", "cpu_baseline"):
+        if k in line:
+            result[k] = line[k]
+    del head
+    if world == 1 and args.extra:
+        per = {}
+        for name in args.extra.split(","):
+            name = name.strip()
+            if not name or name == args.workload:
+                continue
+            torch.cuda.empty_cache()
+            r = measure(wl.WORKLOADS[name], args, dev, timer, cpu_leg_seconds=0.0)
+            per[name] = summarise(r)
+            del r
+        result["per_workload"] = per
+    if world == 1 and args.loops:
+        torch.cuda.empty_cache()
+        result["decode_loop"] = {name: decode_loop(wl.WORKLOADS[name], dev, timer)
+                                 for name in args.loops.split(",") if name}
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -381,32 +578,103 @@ def oracle_sample(w, x, heads):
     return {n: wl.to_oracle(t) for n, t in sub.items()}, w.replace(B=1, Hkv=heads, Hq=heads * g)
 
 
-def cpu_baseline(w, x, seconds=15.0, heads=None, single_seconds=5.0):
-    """The oracle as it stands, on this host's cores, over a bounded sample of
-    the workload (the first KV head(s) of sequence 0), repeated for ~seconds;
-    then the same sample on one core for ~single_seconds."""
+def _swaps(ora_scores, ora_sel, gpu_sel, k):
+    """Selection of each sampled head against the oracle's: exact, or
+    differing only by swaps among spans within 1e-3 relative of the oracle's
+    k-th score.  Returns (swaps, ok)."""
+    import numpy as np
+    swaps, ok = 0, True
+    for idx in np.ndindex(ora_sel.shape[:2]):
+        sc = ora_scores[idx]
+        keff = min(k, sc.size)
+        g = gpu_sel[idx]
+        ok &= bool((g[keff:] == -1).all() and (np.diff(g[:keff]) > 0).all())
+        O, Gs = set(ora_sel[idx][:keff].tolist()), set(g[:keff].tolist())
+        if O == Gs:
+            continue
+        kth = np.sort(sc)[::-1][keff - 1]
+        for sp in O ^ Gs:
+            ok &= bool(0 <= sp < sc.size and abs(sc[sp] - kth) <= 1e-3 * abs(kth))
+        swaps += len(O - Gs)
+    return swaps, ok
+
+
+def cpu_leg(w, x, gpu_sel, gpu_out, seconds=15.0, single_seconds=0.0, heads=1):
+    """The CPU leg: the oracle as it stands on this host's cores over a
+    bounded sample of the workload (the first KV head of sequence 0).  Its
+    first run also gives the parity of that sample: the GPU's selection
+    against the oracle's (swap rule) and the max-abs output error of the
+    sample's query heads (for a prefill chunk: spans and queries sampled).
+    With seconds > 0 the run repeats for ~seconds (cpu_baseline), then for
+    ~single_seconds on one core."""
+    import numpy as np
+
     import oracle
-    heads = heads or 1
+    oracle.set_threads(host_cores())
+    tol = 1e-4 if w.dtype == "f32" else 2e-2
     xs, ws = oracle_sample(w, x, heads)
     _, sb = step_bytes(ws)
+    g = w.Hq // w.Hkv
+    gsel = gpu_sel[:1, :heads]
+    gout = gpu_out[:1, :heads * g].astype(np.float64)
+    t0 = time.perf_counter()
+    if w.C == 1:
+        ref = oracle.step(**xs, G=ws.G, L=ws.L, S=ws.S, k=ws.k, rope_base=ws.rope_base)
+        swaps, ok = _swaps(ref["scores"], ref["sel"], gsel, w.k)
+        if not np.array_equal(ref["sel"], gsel):
+            ref = oracle.step(**xs, G=ws.G, L=ws.L, S=ws.S, k=ws.k, rope_base=ws.rope_base,
+                              sel=gsel)
+        err = float(np.abs(gout - ref["out"]).max())
+        parity = {"sample": f"sequence 0, KV heads 0..{heads - 1} of {w.Hkv}: every span "
+                            "scored, full selection and output", "swaps": swaps,
+                  "selection_ok": ok, "max_abs": err, "tol": tol, "ok": ok and err <= tol}
+    else:
+        # prefill chunk: the chosen spans with the lowest oracle scores must
+        # not lose to unchosen ones (sampled), and sampled queries' outputs
+        rng = np.random.default_rng(0)
+        mask = np.zeros(max(1, (w.T - w.G - w.L + w.S - 1) // w.S), bool)
+        NS = mask.size if w.T > w.G + w.L else 0
+        ok, swaps = True, 0
+        if NS and w.k:
+            chosen = gsel[0, 0][gsel[0, 0] >= 0]
+            mask[chosen] = True
+            ch, un = np.flatnonzero(mask), np.flatnonzero(~mask)
+            pick = np.concatenate([rng.choice(ch, min(8, ch.size), replace=False),
+                                   rng.choice(un, min(8, un.size), replace=False)])
+            pairs = np.stack([np.zeros_like(pick), pick], 1)
+            sc = oracle.span_scores_list(xs["q"], xs["k_cache"], ws.G, ws.L, ws.S, pairs)
+            sel_sc, un_sc = sc[:min(8, ch.size)], sc[min(8, ch.size):]
+            lo = sel_sc.min() if sel_sc.size else np.inf
+            ok = bool(un_sc.size == 0 or un_sc.max() <= lo + 1e-3 * abs(lo))
+        c_list = sorted({0, w.C - 1, *rng.choice(w.C, 14, replace=False).tolist()})
+        ref = oracle.step(**xs, G=ws.G, L=ws.L, S=ws.S, k=ws.k, rope_base=ws.rope_base,
+                          sel=gsel, c_list=c_list)
+        err = float(np.abs(gout[:, :, c_list] - ref["out"][:, :, c_list]).max())
+        parity = {"sample": f"sequence 0, KV head 0: 16 sampled spans (8 chosen, 8 not) "
+                            f"and {len(c_list)} sampled queries", "swaps": swaps,
+                  "selection_ok": ok, "max_abs": err, "tol": tol, "ok": ok and err <= tol}
+    first = time.perf_counter() - t0
+    out = {"parity": parity}
+    if seconds <= 0 or w.C != 1:
+        return out
 
     def timed(limit):
-        t0 = time.perf_counter()
+        t1 = time.perf_counter()
         n = 0
         while True:
             oracle.step(**xs, G=ws.G, L=ws.L, S=ws.S, k=ws.k, rope_base=ws.rope_base,
                         want_scores=False)
             n += 1
-            if time.perf_counter() - t0 > limit:
+            if time.perf_counter() - t1 > limit:
                 break
-        return (time.perf_counter() - t0) / n, n
+        return (time.perf_counter() - t1) / n, n
 
     cores = oracle.max_threads()
     dt, n = timed(seconds)
-    out = {"value": round(sb / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
-           "kind": "oracle", "sample": f"{w.name}: sequence 0, {heads} of {w.Hkv} KV heads "
-                                       f"({heads * (w.Hq // w.Hkv)} query heads), {n} oracle steps",
-           "sec_per_sample_step": round(dt, 4)}
+    out.update({"value": round(sb / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
+                "kind": "oracle", "sample": f"{w.name}: sequence 0, {heads} of {w.Hkv} KV heads "
+                                            f"({heads * g} query heads), {n} oracle steps",
+                "sec_per_sample_step": round(dt, 4), "first_run_s": round(first, 3)})
     if single_seconds > 0:
         oracle.set_threads(1)
         try:
@@ -436,6 +704,7 @@ def run_reference(args):
     else:
         w_used, heads_total = w, w.Hkv
     import oracle
+    oracle.set_threads(host_cores())
     xs, wsamp = oracle_sample(w_used, x, 1)
     _, sb = step_bytes(wsamp)
     for _ in range(args.warmup):
@@ -462,19 +731,34 @@ def run_reference(args):
     del torch
 
 
+DEFAULT_EXTRA = "tiny_f32_4k,llama3_8b_1m_x4,llama3_8b_prefill_256k,qwen2_1p5b_4m"
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama3_8b_128k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-single-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra", default=DEFAULT_EXTRA,
+                    help="comma-separated workloads measured after the headline one (N=1 only); "
+                         "'' for none")
+    ap.add_argument("--loops", default="tiny_f32_4k,llama3_8b_128k",
+                    help="workloads whose graph-replayed decoding loop is timed (N=1 only)")
+    ap.add_argument("--launch-check", action="store_true",
+                    help="multi-rank plumbing only, on CPU ranks (gloo), no GPU work")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch(args.gpus, sys.argv[1:]))
+    if args.launch_check:
+        run_launch_check(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -199,6 +199,112 @@ REATT_API int reatt_append_kv(const reatt_dims *dims, void *k_cache, void *v_cac
  */
 REATT_API int reatt_selftest_bounded_wait(void *ws, int64_t limit_ns, reatt_stream stream);
 
+/* ---------------------------------------------------------------------------
+ * One sequence's cache split by token ranges over several GPUs ("shards").
+ *
+ * The research-map summary ("Limitations") and the OpenReview reply on W4
+ * ("memory overhead tradeoff", 400K tokens on one GPU) name memory as the
+ * method's only bound: the cache of one sequence can outgrow one GPU.  The
+ * step then runs in three local phases with two small exchanges between
+ * them, which the caller performs (e.g. an all-gather over NCCL):
+ *
+ *   1. reatt_shard_candidates  each shard scores the middle spans it holds
+ *                              and keeps its own top-k (score, span id);
+ *   -- exchange: every shard receives every shard's candidates --
+ *   2. reatt_shard_select      every shard computes the same global top-k
+ *                              from the candidates (the global top-k under
+ *                              the order "score desc, id asc" lies inside
+ *                              the union of the shards' top-k);
+ *   3. reatt_shard_attend      each shard attends over the window rows it
+ *                              holds, at their global window positions, and
+ *                              writes an unnormalised partial (m, l, acc);
+ *   -- exchange: every shard (or one) receives every shard's partial --
+ *   4. reatt_merge_partials    out = sum_r 2^(m_r - M) acc_r /
+ *                                    sum_r 2^(m_r - M) l_r,  M = max_r m_r.
+ *
+ * The result equals reatt_step on the whole cache, up to fp32 rounding order.
+ * dims describe the WHOLE sequence (T = all cached tokens); `shard` says
+ * which rows this GPU holds.  Shard r holds cache rows [t_begin, t_end) of
+ * every (batch, KV head), stored at k_cache[((b*Hkv + h)*rows_cap + t -
+ * t_begin)*d] (rows_cap = 0 means t_end - t_begin).  The shards, in rank
+ * order, cover [0, T) without gaps; a boundary inside the middle must fall on
+ * a span boundary (G + multiple of S); exactly one shard owns the current
+ * tokens (owns_current = 1).  reatt_shard_plan makes such a split.  dims->T_cap
+ * is ignored by these calls.  Span scoring of a shard with C > 1 runs on CUDA
+ * cores (the tensor-core prefill scan is not used for shards).
+ * --------------------------------------------------------------------------- */
+typedef struct {
+    int64_t t_begin;        /* first cached token (whole-sequence index) held here  */
+    int64_t t_end;          /* one past the last                                     */
+    int64_t rows_cap;       /* rows allocated per (b, KV head); 0 = t_end - t_begin   */
+    int32_t owns_current;   /* 1 on exactly one shard: it attends the current tokens  */
+    int32_t reserved;       /* 0                                                     */
+} reatt_shard;
+
+/* Splits [0, T) into n (1 <= n <= 1024) contiguous shards that hold nearly
+ * equal numbers of middle spans (boundaries on span boundaries; the global
+ * tokens go with shard 0, the local ones with the last shard, which also owns
+ * the current tokens).  shards: n entries, written on success. */
+REATT_API int reatt_shard_plan(const reatt_dims *dims, int32_t n, reatt_shard *shards);
+
+/* Bytes of device workspace the shard calls of this shard need with
+ * n_shards shards (a multiple of 256).  The status word sits at offset 0, as
+ * in every workspace (reatt_workspace_status reads it). */
+REATT_API int reatt_shard_workspace_bytes(const reatt_dims *dims, const reatt_shard *shard,
+                                          int32_t n_shards, size_t *bytes);
+
+/*
+ * Phase 1 (decoding pseudocode: score = query . key[global:-local]^T,
+ * idx_recall = score.topk, restricted to the spans this shard holds).  For
+ * each (b, h): the min(k, NS_shard) best of this shard's middle spans (ties
+ * to the lower id), as whole-sequence span ids in ascending order with their
+ * fp32 scores; the remaining entries are (-inf, -1).
+ *   q [B,Hq,C,d]; k_cache: this shard's rows; cand_score float [B,Hkv,k];
+ *   cand_id int32 [B,Hkv,k].
+ */
+REATT_API int reatt_shard_candidates(const reatt_dims *dims, const reatt_shard *shard,
+                                     const void *q, const void *k_cache, float *cand_score,
+                                     int32_t *cand_id, void *ws, reatt_stream stream);
+
+/*
+ * Phase 2: the global top-k from every shard's candidates.
+ *   cand_score_all float [n_shards, B, Hkv, k], cand_id_all int32 [n_shards,
+ *   B, Hkv, k] (shard r's phase-1 output at index r, shards in token order)
+ *   -> sel int32 [B, Hkv, k]: ascending span ids, -1 padded, exactly what
+ *   reatt_topk gives on the whole sequence's span scores.
+ */
+REATT_API int reatt_shard_select(const reatt_dims *dims, int32_t n_shards,
+                                 const float *cand_score_all, const int32_t *cand_id_all,
+                                 int32_t *sel, void *ws, reatt_stream stream);
+
+/*
+ * Phase 3 (decoding pseudocode: attention over global ++ recalled ++ local;
+ * "Approach": RoPE after the concatenation): the window rows this shard
+ * holds (its global rows, its chosen spans, its local rows, the current
+ * tokens if it owns them), each rotated at its position in the whole
+ * window, against the queries rotated at W-C+c, causal, scale 1/sqrt(d).
+ * Writes this shard's partial per query row (b, j, c):
+ *   part_ml [B,Hq,C] float2 (m, l): m = max over visible keys of the logit
+ *   times log2(e) (-inf when the shard holds no visible key), l = sum of
+ *   2^(logit*log2(e) - m);
+ *   part_acc [B,Hq,C,d] float: sum of 2^(logit*log2(e) - m) * v.
+ * sel: the phase-2 selection.  k_cur/v_cur are read only by the shard that
+ * owns the current tokens (others may pass them too; NULL is allowed there).
+ */
+REATT_API int reatt_shard_attend(const reatt_dims *dims, const reatt_shard *shard,
+                                 const void *q, const void *k_cache, const void *v_cache,
+                                 const void *k_cur, const void *v_cur, const int32_t *sel,
+                                 void *part_ml, float *part_acc, void *ws, reatt_stream stream);
+
+/*
+ * Phase 4: the log-sum-exp merge of n_parts partials (n_parts >= 1):
+ *   part_ml_all [n_parts,B,Hq,C] float2, part_acc_all [n_parts,B,Hq,C,d]
+ *   -> out [B,Hq,C,d] float32.  A row that no part sees is written as 0.
+ */
+REATT_API int reatt_merge_partials(const reatt_dims *dims, int32_t n_parts,
+                                   const void *part_ml_all, const float *part_acc_all,
+                                   float *out, reatt_stream stream);
+
 /*
  * reatt_step without a caller-supplied workspace.  The pages have no
  * counterpart to this call; it exists for callers that cannot allocate device

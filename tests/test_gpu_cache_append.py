@@ -60,11 +60,12 @@ def _rand(shape, gen, dtype=torch.bfloat16, scale=1.0):
 
 
 def test_chunked_prefill_with_append(R, ora):
-    """The pages' prefill: a first chunk of G+L tokens, then fixed chunks; each
-    chunk attends over the cache built so far (span selection on its middle)
-    and is then appended."""
+    """The pages' prefill: a first chunk of G+L tokens, then chunks of 512
+    tokens (chunk_size=512 in the OpenReview discussion's NIAH settings) and
+    a shorter last one; each chunk attends over the cache built so far (span
+    selection on its middle) and is then appended."""
     B, Hq, Hkv, dh, G, L, S, k, base = 1, 8, 2, 128, 32, 256, 32, 8, 5e5
-    chunks = [G + L] + [256] * 5
+    chunks = [G + L] + [512] * 4 + [300]
     P = sum(chunks)
     gen = torch.Generator().manual_seed(70)
     q_all = _rand((B, Hq, P, dh), gen)

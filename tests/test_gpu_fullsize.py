@@ -1,7 +1,8 @@
 """Parity at the full workload sizes, in the launch configuration the
 benchmark times.  Where the oracle cannot afford every output (the 1M x 4
-batch, the 2048-query prefill chunk) it checks sampled sequences, spans and
-queries, plus properties that hold at any size."""
+batch, the 2048-query prefill chunk) it checks whole sequences or whole KV
+heads in full and samples the rest (spans, queries), plus properties that
+hold at any size."""
 import numpy as np
 import pytest
 import torch
@@ -61,18 +62,38 @@ def test_long_decode(R, ora, name):
 
 
 def test_llama3_8b_prefill_chunk(R, ora):
-    """2048-query chunk over a 256K cache: sampled span scores (the lowest
-    chosen and highest unchosen by GPU score, plus random ones), the
-    selection property on them, and sampled query outputs."""
+    """2048-query chunk over a 256K cache.
+
+    * KV heads 0 and 5: the oracle scores every one of their 8,063 spans
+      (max over the whole chunk's queries, the pages' prefill score), and the
+      GPU's scores and selection of those heads meet the full bars: scores
+      within 2e-5 of the head's max |score|, selection exact up to the swap
+      rule.
+    * The other heads: sampled spans (the lowest chosen and highest unchosen
+      by GPU score, plus random ones) and the selection property on them.
+    * Outputs of 64 queries touching all 16 query tiles of 128 (the first
+      and last query of every tile plus 32 random ones), all 32 query heads."""
     w = wl.WORKLOADS["llama3_8b_prefill_256k"]
     x = _device_inputs(w)
     d = R.dims_of(w)
     gpu = parity.run_all(R, d, {n: x[n] for n in parity.NAMES})
     xh = parity.host_inputs(x)
+    g = w.Hq // w.Hkv
+    full_heads = (0, 5)
+    for h in full_heads:
+        sub = {"q": xh["q"][:, h * g:(h + 1) * g], "k_cache": xh["k_cache"][:, h:h + 1]}
+        oscore = ora.span_scores(sub["q"], sub["k_cache"], w.G, w.L, w.S)   # [1, 1, NS]
+        osel = ora.topk(oscore[0, 0], w.k)[None, None]
+        parity.check_scores(gpu["span_scores"][:, h:h + 1], oscore)
+        for key in ("sel_step", "sel"):
+            swaps = parity.check_selection(oscore, osel, gpu[key][:, h:h + 1], w.k)
+            print("head", h, key, "swaps", swaps)
     rng = np.random.default_rng(1)
     NS = gpu["span_scores"].shape[-1]
     pairs, groups = [], []
     for h in range(w.Hkv):
+        if h in full_heads:
+            continue
         sc = gpu["span_scores"][0, h]
         chosen = gpu["sel_step"][0, h]
         mask = np.zeros(NS, bool)
@@ -92,11 +113,17 @@ def test_llama3_8b_prefill_chunk(R, ora):
     assert np.abs(gscore - oscore).max() <= parity.SCORE_RTOL * scale
     groups = np.array(groups)
     for h in range(w.Hkv):
+        if h in full_heads:
+            continue
         m = pairs[:, 0] == h
         lo = oscore[m & groups].min()
         hi = oscore[m & ~groups].max()
         assert hi <= lo + parity.SWAP_REL * abs(lo), (h, lo, hi)
-    c_list = [0, 1, 511, 1024, 2046, 2047]
+    tiles = np.arange(0, w.C, 128)
+    edges = np.concatenate([tiles, tiles + 127])
+    rest = np.setdiff1d(np.arange(w.C), edges)
+    c_list = np.sort(np.concatenate([edges, rng.choice(rest, 32, replace=False)])).tolist()
+    assert len(c_list) == 64 and len({c // 128 for c in c_list}) == w.C // 128
     for key in ("sel_step", "sel"):
         out_key = "out_step" if key == "sel_step" else "out"
         err = parity.check_outputs(ora, xh, gpu[key], gpu[out_key], w, c_list=c_list)

@@ -104,6 +104,9 @@ inline uint8_t *at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + o
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? REATT_OK : REATT_ECUDA; }
 
 }  // namespace
+
+int geom_of(const reatt_dims *d, Geom *g) { return make_geom(d, g); }
+
 }  // namespace reatt
 
 using namespace reatt;

@@ -36,11 +36,17 @@ inline bool geo_is_bf16(const Geom &g) { return g.dtype == REATT_BF16; }
 
 int num_sms();
 
+// Checked geometry of a call (host argument checks of the C ABI).
+int geom_of(const reatt_dims *d, Geom *g);
+
 // span scoring: scratch holds the fp32 summed queries when C > 1; rope_tab
-// (nullable, decode only) is filled with the step's RoPE table on the side
+// (nullable, decode only) is filled with the step's RoPE table on the side;
+// allow_tc = false keeps C > 1 off the tensor-core scan (its tensor maps need
+// the cache's own base address)
 size_t score_spans_ws_bytes(const Geom &geo);
 cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, float *scores,
-                               void *ws, void *scratch, float2 *rope_tab, cudaStream_t st);
+                               void *ws, void *scratch, float2 *rope_tab, cudaStream_t st,
+                               bool allow_tc = true);
 
 // prefill span scoring on tcgen05 (bf16, C > 1, S divides 32)
 bool prefill_tc_eligible(const Geom &geo);
@@ -63,6 +69,10 @@ size_t topk_ws_bytes(const Geom &geo);
 int topk_selecting_ctas(const Geom &geo);   // CTAs of the first top-k launch that select
 cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void *scratch,
                         uint32_t *zero_words, int nzero, float2 *rope_tab, cudaStream_t st);
+// top-k of candidate lists: per (b, h), ncand order codes and span ids (in
+// ascending id order; code 0 = empty) -> the min(k, NS) best ids, ascending
+cudaError_t launch_topk_merge(const Geom &geo, const uint32_t *codes, const int32_t *ids,
+                              int32_t *sel, int ncand, cudaStream_t st);
 
 // current tokens' K/V rows -> cache rows [T, T + C) (caches of Ts rows per head)
 cudaError_t launch_append(const Geom &geo, void *k_cache, void *v_cache, const void *k_cur,

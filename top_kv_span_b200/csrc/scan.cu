@@ -455,7 +455,8 @@ size_t score_spans_ws_bytes(const Geom &geo)
 }
 
 cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, float *scores,
-                               void *ws, void *scratch, float2 *rope_tab, cudaStream_t st)
+                               void *ws, void *scratch, float2 *rope_tab, cudaStream_t st,
+                               bool allow_tc)
 {
     if (int64_t(geo.B) * geo.Hkv * geo.NS == 0) return cudaSuccess;
     if (geo.C == 1) {
@@ -467,7 +468,7 @@ cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, f
                                 : launch_decode<float, 64>(geo, q, kc, scores, ws, rope_tab, st);
     }
     if (rope_tab) return cudaErrorInvalidValue;   // only the decode scan writes the table
-    if (prefill_tc_eligible(geo))   // tensor-core contraction (tcgen05 / TMEM)
+    if (allow_tc && prefill_tc_eligible(geo))   // tensor-core contraction (tcgen05 / TMEM)
         return launch_prefill_tc(geo, q, kc, scores, ws, scratch, st);
     float *qsum = static_cast<float *>(scratch);
     if (geo.d == 128)

@@ -460,6 +460,15 @@ TopkPlan topk_plan(const Geom &geo)
 
 }  // namespace
 
+cudaError_t launch_topk_merge(const Geom &geo, const uint32_t *codes, const int32_t *ids,
+                              int32_t *sel, int ncand, cudaStream_t st)
+{
+    if (geo.k == 0) return cudaSuccess;
+    topk_merge_kernel<<<unsigned(geo.B * geo.Hkv), kTopkThreads, 0, st>>>(geo, codes, ids, sel,
+                                                                          ncand);
+    return cudaGetLastError();
+}
+
 int topk_selecting_ctas(const Geom &geo)
 {
     return geo.k == 0 ? 0 : geo.B * geo.Hkv * topk_plan(geo).nslices;

@@ -21,7 +21,9 @@ F32, BF16 = 0, 1
 EXPORTS = ["reatt_status_string", "reatt_num_spans", "reatt_window_max", "reatt_workspace_bytes",
            "reatt_workspace_status", "reatt_score_spans", "reatt_topk", "reatt_gather_rope",
            "reatt_attend", "reatt_step", "reatt_append_kv", "reatt_selftest_bounded_wait",
-           "reatt_step_fixed_scratch"]
+           "reatt_step_fixed_scratch", "reatt_shard_plan", "reatt_shard_workspace_bytes",
+           "reatt_shard_candidates", "reatt_shard_select", "reatt_shard_attend",
+           "reatt_merge_partials"]
 
 
 class reatt_dims(ctypes.Structure):
@@ -30,6 +32,12 @@ class reatt_dims(ctypes.Structure):
                 ("L", ctypes.c_int32), ("S", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("T", ctypes.c_int64), ("rope_base", ctypes.c_double),
                 ("T_cap", ctypes.c_int64)]
+
+
+class reatt_shard(ctypes.Structure):
+    _fields_ = [("t_begin", ctypes.c_int64), ("t_end", ctypes.c_int64),
+                ("rows_cap", ctypes.c_int64), ("owns_current", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class ReattError(RuntimeError):
@@ -58,6 +66,14 @@ lib.reatt_step.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.reatt_step_fixed_scratch.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.reatt_selftest_bounded_wait.argtypes = [_vp, ctypes.c_int64, _vp]
 lib.reatt_append_kv.argtypes = [_dp, _vp, _vp, _vp, _vp, _vp]
+_sp = ctypes.POINTER(reatt_shard)
+lib.reatt_shard_plan.argtypes = [_dp, ctypes.c_int32, _sp]
+lib.reatt_shard_workspace_bytes.argtypes = [_dp, _sp, ctypes.c_int32,
+                                            ctypes.POINTER(ctypes.c_size_t)]
+lib.reatt_shard_candidates.argtypes = [_dp, _sp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.reatt_shard_select.argtypes = [_dp, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp]
+lib.reatt_shard_attend.argtypes = [_dp, _sp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.reatt_merge_partials.argtypes = [_dp, ctypes.c_int32, _vp, _vp, _vp, _vp]
 for _name in EXPORTS[1:]:
     getattr(lib, _name).restype = ctypes.c_int
 
@@ -199,6 +215,59 @@ def reatt_step_fixed_scratch(dims, q, k_cache, v_cache, k_cur, v_cur, sel_out, o
                                       _stream(stream))
     if check:
         _check(rc, "reatt_step_fixed_scratch")
+    return rc
+
+
+def reatt_shard_plan(dims, n):
+    """n contiguous shards of the sequence's tokens (list of reatt_shard)."""
+    arr = (reatt_shard * int(n))()
+    _check(lib.reatt_shard_plan(ctypes.byref(dims), int(n), arr), "reatt_shard_plan")
+    return list(arr)
+
+
+def reatt_shard_workspace_bytes(dims, shard, n_shards) -> int:
+    v = ctypes.c_size_t()
+    _check(lib.reatt_shard_workspace_bytes(ctypes.byref(dims), ctypes.byref(shard),
+                                           int(n_shards), ctypes.byref(v)),
+           "reatt_shard_workspace_bytes")
+    return v.value
+
+
+def reatt_shard_candidates(dims, shard, q, k_cache, cand_score, cand_id, ws, stream=None,
+                           check=True):
+    rc = lib.reatt_shard_candidates(ctypes.byref(dims), ctypes.byref(shard), _ptr(q),
+                                    _ptr(k_cache), _ptr(cand_score), _ptr(cand_id), _ptr(ws),
+                                    _stream(stream))
+    if check:
+        _check(rc, "reatt_shard_candidates")
+    return rc
+
+
+def reatt_shard_select(dims, n_shards, cand_score_all, cand_id_all, sel, ws, stream=None,
+                       check=True):
+    rc = lib.reatt_shard_select(ctypes.byref(dims), int(n_shards), _ptr(cand_score_all),
+                                _ptr(cand_id_all), _ptr(sel), _ptr(ws), _stream(stream))
+    if check:
+        _check(rc, "reatt_shard_select")
+    return rc
+
+
+def reatt_shard_attend(dims, shard, q, k_cache, v_cache, k_cur, v_cur, sel, part_ml, part_acc,
+                       ws, stream=None, check=True):
+    rc = lib.reatt_shard_attend(ctypes.byref(dims), ctypes.byref(shard), _ptr(q), _ptr(k_cache),
+                                _ptr(v_cache), _ptr(k_cur), _ptr(v_cur), _ptr(sel),
+                                _ptr(part_ml), _ptr(part_acc), _ptr(ws), _stream(stream))
+    if check:
+        _check(rc, "reatt_shard_attend")
+    return rc
+
+
+def reatt_merge_partials(dims, n_parts, part_ml_all, part_acc_all, out, stream=None,
+                         check=True):
+    rc = lib.reatt_merge_partials(ctypes.byref(dims), int(n_parts), _ptr(part_ml_all),
+                                  _ptr(part_acc_all), _ptr(out), _stream(stream))
+    if check:
+        _check(rc, "reatt_merge_partials")
     return rc
 
 
