@@ -43,8 +43,11 @@ METRIC = "ReAttention step latency (µs) and KV-scan GB/s vs HBM peak at 128K–
 PROFILE_SUMMARY = {
     "llama3_8b_128k": os.path.join(ROOT, "profiles", "scan_decode_llama3_8b_128k.md"),
     "llama3_8b_prefill_256k": os.path.join(ROOT, "profiles",
-                                           "scan_prefill_tc_llama3_8b_prefill_256k.md"),
+                                           "scan_prefill_tc_llama3_8b_prefill_64k.md"),
+    "qwen2_1p5b_4m": os.path.join(ROOT, "profiles", "scan_decode_qwen2_1p5b_4m.md"),
 }
+# key of the traffic line in a summary (a smaller capture scaled to the workload)
+PROFILE_KEY = {"llama3_8b_prefill_256k": "traffic_bytes_per_launch_256k:"}
 
 
 def step_bytes(w):
@@ -66,10 +69,11 @@ def read_traffic(workload):
     path = PROFILE_SUMMARY.get(workload)
     if path is None:
         return None
+    key = PROFILE_KEY.get(workload, "traffic_bytes_per_launch:")
     try:
         with open(path) as f:
             for line in f:
-                if line.startswith("traffic_bytes_per_launch:"):
+                if line.startswith(key):
                     v = line.split(":", 1)[1].strip()
                     return None if v in ("null", "") else float(v)
     except OSError:

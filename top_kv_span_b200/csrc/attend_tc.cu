@@ -17,13 +17,17 @@
 // 128-row query block:
 //   warp 0   TMA producer: the query block once, then 64-key tiles of K (hi,
 //            lo) and V^T in a 2-stage ring (128B swizzle, no multicast)
-//   warp 1   TMEM allocation; one thread issues S(j) into one of two TMEM
-//            S buffers, then O += P(j-1).V(j-1) into the TMEM O accumulator
-//   warps 2-5 softmax: one thread per query row reads its S row from TMEM,
-//            masks (causal, window end), keeps a running reference max that
-//            moves (and rescales O in TMEM) only when the row max grows by
-//            more than 2^8, writes P in the swizzled operand layout into one
-//            of two P buffers, and finally divides O by the row sum.
+//   warp 1   TMEM allocation; one thread issues, whichever is ready, S(j)
+//            into one of two TMEM S buffers and O += P(j).V(j) into the TMEM
+//            O accumulator (S never waits behind a P.V)
+//   warps 2-9 softmax: two warps per TMEM lane group, one per 32-column half
+//            of the S tile; a thread owns one query row's half: it reads its
+//            32 S values from TMEM, masks (causal, window end), trades its
+//            half-row max with the partner warp (a named barrier per pair),
+//            keeps a running reference max that moves (and rescales its half
+//            of O in TMEM) only when the row max grows by more than 2^8,
+//            writes its half of P in the swizzled operand layout into one of
+//            two P buffers, and finally divides its half of O by the row sum.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -40,7 +44,8 @@ namespace {
 
 using namespace tc;
 
-constexpr int kFaThreads = 6 * 32;
+constexpr int kFaSoftWarps = 8;          // two per TMEM lane group
+constexpr int kFaThreads = (2 + kFaSoftWarps) * 32;
 constexpr int kQRows = 128;   // query rows per CTA (TMEM lanes)
 constexpr int kKeyTile = 64;  // keys per S tile (S columns)
 constexpr float kRescaleLog2 = 8.f;
@@ -238,8 +243,8 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
             mbar_init(&vfull[s], 1);
             mbar_init(&vempty[s], 1);
             mbar_init(&sfull[s], 1);
-            mbar_init(&sempty[s], 4);
-            mbar_init(&pfull[s], 4);     // P buffer s written (one arrival per softmax warp)
+            mbar_init(&sempty[s], kFaSoftWarps);
+            mbar_init(&pfull[s], kFaSoftWarps);   // P buffer s written (one arrival per softmax warp)
             mbar_init(&pvdone[s], 1);    // P(s).V done: buffer s free again
         }
         mbar_init(done, 1);
@@ -321,15 +326,17 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
             bool ok = !aborted() && mbar_wait_bounded(qfull, 0, kWaitLimitNs);
             if (!ok) fail();
             tc_fence_after();
-            for (int j = 0; ok && j <= nt; ++j) {
-                if (j < nt) {   // S(j) = Q.K(j)^T (three hi/lo products)
-                    const int s = j & 1;
-                    if (aborted() || !mbar_wait_bounded(&kfull[s], (j >> 1) & 1, kWaitLimitNs) ||
-                        (j >= 2 && !mbar_wait_bounded(&sempty[s], ((j >> 1) - 1) & 1, kWaitLimitNs))) {
-                        fail();
-                        ok = false;
-                        break;
-                    }
+            // Whichever is ready: S(js) as soon as K(js) has landed and the
+            // softmax has read S buffer js&1 (S(js-2)), P(jp).V(jp) as soon as
+            // the softmax has written P(jp).  S never waits for a P.V, so the
+            // tensor cores compute the next tiles' S while the softmax works.
+            int js = 0, jp = 0;
+            uint64_t t_last = global_ns();
+            while (ok && jp < nt) {
+                bool progressed = false;
+                if (js < nt && mbar_test(&kfull[js & 1], (js >> 1) & 1) &&
+                    (js < 2 || mbar_test(&sempty[js & 1], ((js >> 1) - 1) & 1))) {
+                    const int s = js & 1;   // S(js) = Q.K(js)^T (three hi/lo products)
                     tc_fence_after();
                     const uint8_t *kst = smem + Sm::oK + s * 2 * Sm::kK;
                     const uint32_t d_s = tmem_base + uint32_t(s * kKeyTile);
@@ -346,15 +353,12 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                     }
                     tc_commit(&sfull[s]);
                     tc_commit(&kempty[s]);
+                    ++js;
+                    progressed = true;
                 }
-                if (j >= 1) {   // O += P(j-1).V(j-1) (hi and lo P)
-                    const int jj = j - 1, s = jj & 1;
-                    if (aborted() || !mbar_wait_bounded(&pfull[s], (jj >> 1) & 1, kWaitLimitNs) ||
-                        !mbar_wait_bounded(&vfull[s], (jj >> 1) & 1, kWaitLimitNs)) {
-                        fail();
-                        ok = false;
-                        break;
-                    }
+                if (jp < js && mbar_test(&pfull[jp & 1], (jp >> 1) & 1) &&
+                    mbar_test(&vfull[jp & 1], (jp >> 1) & 1)) {
+                    const int s = jp & 1;   // O += P(jp).V(jp)
                     tc_fence_after();
                     const uint32_t d_o = tmem_base + 128u;
                     const uint8_t *vst = smem + Sm::oV + s * Sm::kV;
@@ -362,70 +366,91 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                     for (int ks = 0; ks < PS; ++ks) {
                         const uint64_t pd = sw128_desc(smem + Sm::oP + s * Sm::kP) + uint64_t(ks * 2);
                         const uint64_t vd = sw128_desc(vst) + uint64_t(ks * 2);
-                        tc_mma(d_o, pd, vd, id_o, (jj > 0 || ks > 0) ? 1u : 0u);
+                        tc_mma(d_o, pd, vd, id_o, (jp > 0 || ks > 0) ? 1u : 0u);
                     }
                     tc_commit(&pvdone[s]);
                     tc_commit(&vempty[s]);
+                    ++jp;
+                    progressed = true;
+                }
+                if (progressed) {
+                    t_last = global_ns();
+                } else if (aborted() || global_ns() - t_last > kWaitLimitNs) {
+                    fail();
+                    ok = false;
+                } else {
+                    __nanosleep(32);   // leave the issue slots to the softmax warps
                 }
             }
             tc_commit(done);
             if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) fail();
         }
     } else {
-        // ------------------------------------------------ softmax warps (one query row each)
-        const int quad = warp & 3;
+        // ------------------------------------------------ softmax warps (half a query row each)
+        // The two warps of a lane group keep identical row state (same
+        // maxima, same decisions) and leave the loop together: every tile
+        // they trade their half-row maxima and their status through
+        // shared memory (double-buffered by tile parity) across one named
+        // barrier of the pair.
+        __shared__ float xmax[2][4][2][32], xsum[4][2][32];
+        __shared__ int xok[2][4][2];
+        const int quad = warp & 3;               // TMEM lanes this warp may access
+        const int half = (warp - 2) >> 2;        // S columns [32*half, 32*half + 32)
         const int row = quad * 32 + lane;
         const uint32_t lane_base = tmem_base + (uint32_t(quad * 32) << 16);
         const bool live = row < nrows;
         const int64_t qpos = live ? qpos0 + (r0 + row) % geo.C : -1;
         // last key this row sees (window end and causal limit); -1: none
         const int row_lim = live ? int((kend - 1 < qpos) ? kend - 1 : qpos) : -1;
+        auto pair_sync = [&] { named_sync(1 + quad, 64); };
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         uint8_t *pbuf = smem + Sm::oP;
+        constexpr int HC = kKeyTile / 2;         // columns per warp
         for (int j = 0; j < nt; ++j) {
             const int s = j & 1;
-            bool got = !aborted() && mbar_wait_bounded(&sfull[s], (j >> 1) & 1, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, got)) {
-                if (lane == 0) fail();
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            float sv[kKeyTile];
-            {
-                float t[32];
-                tmem_ld32(lane_base + uint32_t(s * kKeyTile), t);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sv[i] = t[i];
-                tmem_ld32(lane_base + uint32_t(s * kKeyTile + 32), t);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sv[32 + i] = t[i];
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sempty[s]);
-            // keys past this row's limit (window end, causal) are masked;
-            // tiles wholly inside the limit skip the per-key test
-            float mx = -INFINITY;
-            const int kb = j * kKeyTile;
-            if (kb + kKeyTile - 1 <= row_lim) {
-#pragma unroll
-                for (int i = 0; i < kKeyTile; ++i) mx = fmaxf(mx, sv[i]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < kKeyTile; ++i) {
-                    if (kb + i > row_lim) sv[i] = -INFINITY;
-                    mx = fmaxf(mx, sv[i]);
-                }
-            }
-            // P buffer j&1 is free once P(j-2).V(j-2) has completed
-            if (j >= 2) {
-                got = !aborted() && mbar_wait_bounded(&pvdone[s], ((j - 2) >> 1) & 1, kWaitLimitNs);
+            if (ok) {
+                const bool got = !aborted() && mbar_wait_bounded(&sfull[s], (j >> 1) & 1, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, got)) {
                     if (lane == 0) fail();
                     ok = false;
-                    break;
+                }
+            }
+            float sv[HC];
+            float mx = -INFINITY;
+            if (ok) {
+                tc_fence_after();
+                tmem_ld32(lane_base + uint32_t(s * kKeyTile + half * HC), sv);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sempty[s]);
+                // keys past this row's limit (window end, causal) are masked;
+                // halves wholly inside the limit skip the per-key test
+                const int kb = j * kKeyTile + half * HC;
+                if (kb + HC - 1 <= row_lim) {
+#pragma unroll
+                    for (int i = 0; i < HC; ++i) mx = fmaxf(mx, sv[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < HC; ++i) {
+                        if (kb + i > row_lim) sv[i] = -INFINITY;
+                        mx = fmaxf(mx, sv[i]);
+                    }
+                }
+            }
+            xmax[s][quad][half][lane] = mx;
+            if (lane == 0) xok[s][quad][half] = ok ? 1 : 0;
+            pair_sync();
+            if (!xok[s][quad][0] || !xok[s][quad][1]) break;   // both warps leave together
+            mx = fmaxf(mx, xmax[s][quad][half ^ 1][lane]);
+            // P buffer j&1 is free once P(j-2).V(j-2) has completed
+            if (j >= 2) {
+                const bool got =
+                    !aborted() && mbar_wait_bounded(&pvdone[s], ((j - 2) >> 1) & 1, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) fail();
+                    ok = false;   // reported at the next exchange; no P or O access now
+                    continue;
                 }
                 tc_fence_after();
             }
@@ -440,19 +465,19 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
             if (j >= 1 && __any_sync(0xffffffffu, move && fac != 1.f)) {
                 // O is quiescent once P(j-1).V(j-1) has completed (P(j).V is
                 // issued only after this tile's P is written)
-                got = !aborted() &&
-                      mbar_wait_bounded(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, kWaitLimitNs);
+                const bool got = !aborted() &&
+                                 mbar_wait_bounded(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, got)) {
                     if (lane == 0) fail();
                     ok = false;
-                    break;
+                    continue;
                 }
                 tc_fence_after();
-                // rescale this row of O in TMEM (warp-collective accesses)
+                // rescale this row's half of O in TMEM (warp-collective accesses)
 #pragma unroll
-                for (int cb = 0; cb < D / 32; ++cb) {
+                for (int cb = 0; cb < D / 64; ++cb) {
                     float o[32];
-                    const uint32_t ta = lane_base + 128u + uint32_t(cb * 32);
+                    const uint32_t ta = lane_base + 128u + uint32_t(half * (D / 2) + cb * 32);
                     tmem_ld32(ta, o);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] *= fac;
@@ -460,12 +485,13 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                 }
             }
             // P = exp2(S - m_ref) <= 2^8 as fp16 (11-bit significand), 128B-
-            // swizzled K-major rows of buffer j&1
+            // swizzled K-major rows of buffer j&1; this warp writes chunks
+            // [4*half, 4*half + 4) of the row
             const bool any_key = m_ref != -INFINITY;
             uint8_t *pw = pbuf + s * Sm::kP + row * 128;
             float rs = 0.f;
 #pragma unroll
-            for (int c = 0; c < kKeyTile / 8; ++c) {
+            for (int c = 0; c < HC / 8; ++c) {
                 uint32_t hw[4];
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
@@ -477,7 +503,8 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                     const __half2 hv = __floats2half2_rn(p0, p1);
                     hw[e / 2] = *reinterpret_cast<const uint32_t *>(&hv);
                 }
-                *reinterpret_cast<uint4 *>(pw + (c ^ (row & 7)) * 16) =
+                const int ch = half * (HC / 8) + c;
+                *reinterpret_cast<uint4 *>(pw + (ch ^ (row & 7)) * 16) =
                     make_uint4(hw[0], hw[1], hw[2], hw[3]);
             }
             l += rs;
@@ -485,6 +512,11 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
             __syncwarp();
             if (lane == 0) mbar_arrive(&pfull[s]);
         }
+        // row sum over both halves (both warps reach this barrier: they leave
+        // the loop at the same tile or finish it)
+        xsum[quad][half][lane] = l;
+        pair_sync();
+        l += xsum[quad][half ^ 1][lane];
         if (ok && nt > 0) {
             const bool got = !aborted() &&
                              mbar_wait_bounded(&pvdone[(nt - 1) & 1], ((nt - 1) >> 1) & 1, kWaitLimitNs);
@@ -494,12 +526,12 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
                 tc_fence_after();
                 const int r = r0 + row;
                 const int j = h * geo.g + (live ? r / geo.C : 0), c = live ? r % geo.C : 0;
-                float *dst = fa.out + ((int64_t(b) * geo.Hq + j) * geo.C + c) * D;
+                float *dst = fa.out + ((int64_t(b) * geo.Hq + j) * geo.C + c) * D + half * (D / 2);
                 const float il = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-                for (int cb = 0; cb < D / 32; ++cb) {
+                for (int cb = 0; cb < D / 64; ++cb) {
                     float o[32];
-                    tmem_ld32(lane_base + 128u + uint32_t(cb * 32), o);
+                    tmem_ld32(lane_base + 128u + uint32_t(half * (D / 2) + cb * 32), o);
                     if (live) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)

@@ -82,6 +82,11 @@ WORKLOADS = {
         "llama3_8b_prefill_256k", B=1, Hq=32, Hkv=8, d=128, C=2048, T=262144, G=32, L=4096,
         S=32, k=64, dtype="bf16", rope_base=5e5, seed=1003, n_needles=0, dist="channel",
         description="LLaMA3-8B-shaped bf16 chunked prefill: 2048-query chunk over 256K cache"),
+    "llama3_8b_prefill_64k": Workload(
+        "llama3_8b_prefill_64k", B=1, Hq=32, Hkv=8, d=128, C=2048, T=65536, G=32, L=4096,
+        S=32, k=64, dtype="bf16", rope_base=5e5, seed=1005, n_needles=0, dist="channel",
+        description="the 2048-query prefill chunk over a 64K cache: K+V 268 MB (more than "
+                    "L2), the size full profiler captures of the prefill kernels run on"),
     "qwen2_1p5b_4m": Workload(
         "qwen2_1p5b_4m", B=1, Hq=12, Hkv=2, d=128, C=1, T=4194304, G=32, L=4096, S=32, k=64,
         dtype="bf16", rope_base=1e6, seed=1004, n_needles=5, dist="channel",
