@@ -14,12 +14,14 @@
 //
 // Kernel: one CTA per SM, persistent over (head, 256-token) items: two K tiles
 // of 128 tokens share every query stage, halving the L2 bytes per MMA.
-//   warp 0  : TMA producer (cp.async.bulk.tensor, 128B swizzle, no multicast)
+//   warp 0  : TMA producer (cp.async.bulk.tensor, 128B swizzle, no multicast);
+//             two K stages, so the next item's tiles load while this one runs
 //   warp 1  : TMEM allocation; one thread issues tcgen05.mma (M=128 tokens,
 //             N=128 queries, K=16) per K tile into two accumulator sets in turn
-//   warps 2-5: epilogue -- tcgen05.ld of the accumulator rows (one token row
-//             per thread), max over valid queries, then a segmented warp max
-//             over the span's tokens; only span scores reach global memory.
+//   warps 2-9: epilogue, two warps per TMEM lane group (one per K tile) --
+//             tcgen05.ld of the accumulator rows (one token row per thread),
+//             max over valid queries, then a segmented warp max over the
+//             span's tokens; only span scores reach global memory.
 // Every wait is bounded; a timeout records REATT_ETIMEOUT in the workspace.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -36,11 +38,13 @@ namespace {
 
 using namespace tc;
 
-constexpr int kTcThreads = 6 * 32;   // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kTcEpiWarps = 8;       // two per TMEM lane group: one per K tile
+constexpr int kTcThreads = (2 + kTcEpiWarps) * 32;   // warp 0 TMA, warp 1 MMA, epilogue
 constexpr int kTileM = 128;          // tokens per tile = TMEM lanes
 constexpr int kTiles = 2;            // token tiles per item: each query stage feeds both
 constexpr int kTileN = 128;          // queries per MMA tile = TMEM columns
-constexpr int kQStages = 4;          // query-tile ring
+constexpr int kQStages = 3;          // query-tile ring
+constexpr int kKStages = 2;          // K items: the next item's tiles load during this one
 constexpr uint32_t kTmemCols = 512;  // two accumulator sets of kTiles x 128 columns
 
 struct TcArgs {
@@ -66,10 +70,10 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint8_t *ksm = smem;
-    uint8_t *qsm = smem + kKBytes;
+    uint8_t *qsm = smem + kKStages * kKBytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(qsm + kQStages * kQBytes);
-    uint64_t *kfull = bars, *kempty = bars + 1;
-    uint64_t *qfull = bars + 2, *qempty = qfull + kQStages;
+    uint64_t *kfull = bars, *kempty = bars + kKStages;
+    uint64_t *qfull = kempty + kKStages, *qempty = qfull + kQStages;
     uint64_t *accfull = qempty + kQStages, *accempty = accfull + 2, *done = accempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
     __shared__ int abort_flag;
@@ -77,15 +81,17 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         abort_flag = 0;
-        mbar_init(kfull, 1);
-        mbar_init(kempty, 1);
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(&kfull[s], 1);
+            mbar_init(&kempty[s], 1);
+        }
         for (int s = 0; s < kQStages; ++s) {
             mbar_init(&qfull[s], 1);
             mbar_init(&qempty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&accfull[s], 1);
-            mbar_init(&accempty[s], 4);   // one arrival per epilogue warp
+            mbar_init(&accempty[s], kTcEpiWarps);   // one arrival per epilogue warp
         }
         mbar_init(done, 1);
         mbar_init_fence();
@@ -114,16 +120,18 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 const int64_t bh = it / ta.ntiles;
                 const int tile = int(it % ta.ntiles);
                 const int y = int(bh * geo.Ts + geo.G + int64_t(tile) * kTiles * kTileM);
-                if (kuse > 0 && (aborted() || !mbar_wait_bounded(kempty, (kuse - 1) & 1, kWaitLimitNs))) {
+                const int ks_ = int(kuse % kKStages);
+                const uint32_t kround = kuse / kKStages;
+                if (kround > 0 && (aborted() || !mbar_wait_bounded(&kempty[ks_], (kround - 1) & 1, kWaitLimitNs))) {
                     fail();
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(kfull, kKBytes);
+                mbar_arrive_expect_tx(&kfull[ks_], kKBytes);
                 for (int t = 0; t < kTiles; ++t)
                     for (int bx = 0; bx < NBOX; ++bx)
-                        tma_load_2d(ksm + (t * NBOX + bx) * kBoxBytes, &kmap, 64 * bx,
-                                    y + t * kTileM, kfull);
+                        tma_load_2d(ksm + ks_ * kKBytes + (t * NBOX + bx) * kBoxBytes, &kmap,
+                                    64 * bx, y + t * kTileM, &kfull[ks_]);
                 ++kuse;
                 for (int qt = 0; ok && qt < ta.nqt; ++qt)
                     for (int term = 0; term < ta.nterms; ++term, ++qn) {
@@ -141,8 +149,9 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                                         &qfull[st]);
                     }
             }
-            // drain: the last K load and the last query loads have landed
-            if (kuse > 0 && !mbar_wait_bounded(kfull, (kuse - 1) & 1, kWaitLimitNs)) fail();
+            // drain: the last K loads and the last query loads have landed
+            for (uint32_t m = kuse > kKStages ? kuse - kKStages : 0; m < kuse; ++m)
+                if (!mbar_wait_bounded(&kfull[m % kKStages], (m / kKStages) & 1, kWaitLimitNs)) fail();
             for (uint32_t m = qn > kQStages ? qn - kQStages : 0; m < qn; ++m)
                 if (!mbar_wait_bounded(&qfull[m % kQStages], (m / kQStages) & 1, kWaitLimitNs)) fail();
         }
@@ -152,11 +161,13 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             uint32_t kuse = 0, qn = 0, an = 0;
             bool ok = true;
             for (int64_t it = blockIdx.x; ok && it < ta.items; it += gridDim.x) {
-                if (aborted() || !mbar_wait_bounded(kfull, kuse & 1, kWaitLimitNs)) {
+                const int ks_ = int(kuse % kKStages);
+                if (aborted() || !mbar_wait_bounded(&kfull[ks_], (kuse / kKStages) & 1, kWaitLimitNs)) {
                     fail();
                     break;
                 }
                 ++kuse;
+                const uint8_t *kst = ksm + ks_ * kKBytes;
                 tc_fence_after();
                 for (int qt = 0; ok && qt < ta.nqt; ++qt, ++an) {
                     const int acc = int(an & 1);
@@ -182,7 +193,7 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                             for (int ks = 0; ks < KS; ++ks) {
                                 const int bx = ks / 4, kin = ks % 4;   // box, 32-byte step inside it
                                 const uint64_t adesc =
-                                    sw128_desc(ksm + (t * NBOX + bx) * kBoxBytes) + uint64_t(kin * 2);
+                                    sw128_desc(kst + (t * NBOX + bx) * kBoxBytes) + uint64_t(kin * 2);
                                 const uint64_t bdesc =
                                     sw128_desc(qsm + st * kQBytes + bx * kBoxBytes) + uint64_t(kin * 2);
                                 tc_mma(d_tmem + uint32_t(t * kTileN), adesc, bdesc,
@@ -192,23 +203,23 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     }
                     if (ok) tc_commit(&accfull[acc]);
                 }
-                if (ok) tc_commit(kempty);
+                if (ok) tc_commit(&kempty[ks_]);
             }
             // every MMA issued so far has completed before TMEM is released
             tc_commit(done);
             if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) fail();
         }
     } else {
-        // ------------------------------------------------ epilogue (128 threads)
+        // ------------------------------------------------ epilogue (256 threads)
+        static_assert(kTcEpiWarps == 4 * kTiles, "one warp per lane group and K tile");
         const int quad = warp & 3;              // TMEM lane quadrant of this warp
+        const int t = (warp - 2) >> 2;          // K tile of this warp
         const int row = quad * 32 + lane;       // token row in the tile
         uint32_t an = 0;
         for (int64_t it = blockIdx.x; it < ta.items; it += gridDim.x) {
             const int64_t bh = it / ta.ntiles;
             const int tile = int(it % ta.ntiles);
-            float tokmax[kTiles];
-#pragma unroll
-            for (int t = 0; t < kTiles; ++t) tokmax[t] = -INFINITY;
+            float tokmax = -INFINITY;
             bool ok = true;
             for (int qt = 0; qt < ta.nqt; ++qt, ++an) {
                 const int acc = int(an & 1);
@@ -220,10 +231,17 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     break;
                 }
                 tc_fence_after();
+                const uint32_t taddr = tmem_base + (uint32_t(quad * 32) << 16) +
+                                       uint32_t((acc * kTiles + t) * kTileN);
+                if ((qt + 1) * kTileN <= geo.C) {   // every query of the tile is real
 #pragma unroll
-                for (int t = 0; t < kTiles; ++t) {
-                    const uint32_t taddr = tmem_base + (uint32_t(quad * 32) << 16) +
-                                           uint32_t((acc * kTiles + t) * kTileN);
+                    for (int ch = 0; ch < kTileN / 32; ++ch) {
+                        float v[32];
+                        tmem_ld32(taddr + uint32_t(ch * 32), v);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) tokmax = fmaxf(tokmax, v[j]);
+                    }
+                } else {
 #pragma unroll
                     for (int ch = 0; ch < kTileN / 32; ++ch) {
                         float v[32];
@@ -231,7 +249,7 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                         const int c0 = qt * kTileN + ch * 32;
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            if (c0 + j < geo.C) tokmax[t] = fmaxf(tokmax[t], v[j]);
+                            if (c0 + j < geo.C) tokmax = fmaxf(tokmax, v[j]);
                     }
                 }
                 tc_fence_before();
@@ -240,13 +258,10 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             }
             if (!ok) break;
             // span max: S divides 32, tiles start on span boundaries
-#pragma unroll
-            for (int t = 0; t < kTiles; ++t) {
-                const int64_t moff = (int64_t(tile) * kTiles + t) * kTileM + row;
-                float val = moff < geo.M ? tokmax[t] : -INFINITY;
-                for (int o = 1; o < geo.S; o <<= 1) val = fmaxf(val, __shfl_xor_sync(0xffffffffu, val, o));
-                if (moff < geo.M && (lane % geo.S) == 0) scores[bh * geo.NS + moff / geo.S] = val;
-            }
+            const int64_t moff = (int64_t(tile) * kTiles + t) * kTileM + row;
+            float val = moff < geo.M ? tokmax : -INFINITY;
+            for (int o = 1; o < geo.S; o <<= 1) val = fmaxf(val, __shfl_xor_sync(0xffffffffu, val, o));
+            if (moff < geo.M && (lane % geo.S) == 0) scores[bh * geo.NS + moff / geo.S] = val;
         }
     }
     tc_fence_before();
@@ -360,7 +375,8 @@ cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, fl
     int grid = num_sms();
     if (ta.items < grid) grid = int(ta.items);
     const size_t box = kBoxBytes;
-    const size_t smem = 1024 + (geo.d / 64) * box * (kTiles + kQStages) + (2 + 2 * kQStages + 5) * 8 + 16;
+    const size_t smem = 1024 + (geo.d / 64) * box * (kKStages * kTiles + kQStages) +
+                        (2 * kKStages + 2 * kQStages + 5) * 8 + 16;
     if (geo.d == 128) {
         auto kern = scan_prefill_tc_kernel<128>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
