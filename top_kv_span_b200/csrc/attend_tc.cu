@@ -99,12 +99,6 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
-__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16 &hi, __nv_bfloat16 &lo)
-{
-    hi = __float2bfloat16_rn(x);
-    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-}
-
 // Operand buffers of one call, bf16, per KV head bh:
 //   qh/ql [BH][Rp][D]  rotated queries x log2(e)/sqrt(d), rows >= R zero
 //   kh/kl [BH][Wp][D]  rotated window keys, rows >= W zero
@@ -117,6 +111,26 @@ struct PrepOut {
 
 constexpr int kPrepRows = 64;
 
+// 8 floats -> 8 bf16 (16 bytes)
+__device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8])
+{
+    uint4 w;
+    uint32_t *u = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        u[e] = *reinterpret_cast<const uint32_t *>(&t);
+    }
+    return w;
+}
+__device__ __forceinline__ void unpack8_bf16(const uint4 &w, float (&v)[8])
+{
+    Elem<uint16_t>::unpack(w, v);
+}
+
+// One thread item = 8 consecutive RoPE pairs (dims i0..i0+7 and their
+// partners at +D/2) of one row: 16-byte loads and stores throughout; the
+// cos/sin come from the step's table (the query positions W-C+c are inside it).
 template <int D>
 __global__ void __launch_bounds__(256)
 prefill_prep_kernel(Geom geo, const uint16_t *__restrict__ q, const uint16_t *__restrict__ kc,
@@ -124,45 +138,85 @@ prefill_prep_kernel(Geom geo, const uint16_t *__restrict__ q, const uint16_t *__
                     const uint16_t *__restrict__ vcur, const int32_t *__restrict__ sel,
                     const float2 *__restrict__ tab, PrepOut po)
 {
+    constexpr int NCH = D / 2 / 8;   // 8-pair chunks per row
     __shared__ float vs[kPrepRows][D + 1];
-    __shared__ float2 freq[D / 2];
     pdl_wait();   // the selection and the RoPE table come from the top-k launch
     const int64_t bh = blockIdx.y;
     const int b = int(bh / geo.Hkv), h = int(bh % geo.Hkv);
     const int32_t *sel_bh = sel + bh * geo.k;
     const WinMapTc m = winmap_tc(geo, sel_bh);
-    if (threadIdx.x < D / 2) freq[threadIdx.x] = make_float2(geo.rope_hi[threadIdx.x], geo.rope_lo[threadIdx.x]);
-    __syncthreads();
     const int nkb = po.Wp / kPrepRows;
+    auto rot8 = [&](const uint4 &xw, const uint4 &yw, const float2 *cs, float (&lo)[8],
+                    float (&hi)[8], float scale) {
+        float x[8], y[8];
+        unpack8_bf16(xw, x);
+        unpack8_bf16(yw, y);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            lo[e] = (x[e] * cs[e].x - y[e] * cs[e].y) * scale;
+            hi[e] = (y[e] * cs[e].x + x[e] * cs[e].y) * scale;
+        }
+    };
+    auto split_store = [&](const float (&v)[8], __nv_bfloat16 *dh, __nv_bfloat16 *dl) {
+        float hv[8], lv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            hv[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+            lv[e] = v[e] - hv[e];
+        }
+        *reinterpret_cast<uint4 *>(dh) = pack8_bf16(hv);
+        *reinterpret_cast<uint4 *>(dl) = pack8_bf16(lv);
+    };
     if (int(blockIdx.x) < nkb) {
         // ---- 64 window rows: rotated K hi/lo, V transposed
         const int64_t p0 = int64_t(blockIdx.x) * kPrepRows;
-        for (int x = threadIdx.x; x < kPrepRows * (D / 2); x += blockDim.x) {
-            const int r = x / (D / 2), i = x % (D / 2);
+        for (int x = threadIdx.x; x < kPrepRows * NCH; x += blockDim.x) {
+            const int r = x / NCH, i0 = (x % NCH) * 8;
             const int64_t p = p0 + r;
-            float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+            float k0[8], k1[8], v0[8], v1[8];
             if (p < m.W) {
                 const int64_t off = row_src_tc(geo, m, sel_bh, bh, p, D);
                 const bool cur = (off >> 62) != 0;
                 const int64_t o = off & ~(int64_t(1) << 62);
                 const uint16_t *kr = (cur ? kcur : kc) + o, *vr = (cur ? vcur : vc) + o;
-                const float a = Elem<uint16_t>::one(kr, i), c = Elem<uint16_t>::one(kr, i + D / 2);
-                const float2 cs = tab[p * (D / 2) + i];
-                k0 = a * cs.x - c * cs.y;
-                k1 = c * cs.x + a * cs.y;
-                v0 = Elem<uint16_t>::one(vr, i);
-                v1 = Elem<uint16_t>::one(vr, i + D / 2);
+                const uint4 kx = *reinterpret_cast<const uint4 *>(kr + i0);
+                const uint4 ky = *reinterpret_cast<const uint4 *>(kr + D / 2 + i0);
+                unpack8_bf16(*reinterpret_cast<const uint4 *>(vr + i0), v0);
+                unpack8_bf16(*reinterpret_cast<const uint4 *>(vr + D / 2 + i0), v1);
+                float2 cs[8];
+                const float4 *tr = reinterpret_cast<const float4 *>(tab + p * (D / 2) + i0);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 t4 = tr[e];
+                    cs[2 * e] = make_float2(t4.x, t4.y);
+                    cs[2 * e + 1] = make_float2(t4.z, t4.w);
+                }
+                rot8(kx, ky, cs, k0, k1, 1.f);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) k0[e] = k1[e] = v0[e] = v1[e] = 0.f;
             }
             const int64_t kb = (bh * po.Wp + p) * D;
-            split_bf16(k0, po.kh[kb + i], po.kl[kb + i]);
-            split_bf16(k1, po.kh[kb + i + D / 2], po.kl[kb + i + D / 2]);
-            vs[r][i] = v0;
-            vs[r][i + D / 2] = v1;
+            split_store(k0, po.kh + kb + i0, po.kl + kb + i0);
+            split_store(k1, po.kh + kb + D / 2 + i0, po.kl + kb + D / 2 + i0);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                vs[r][i0 + e] = v0[e];
+                vs[r][D / 2 + i0 + e] = v1[e];
+            }
         }
         __syncthreads();
-        for (int x = threadIdx.x; x < D * kPrepRows; x += blockDim.x) {
-            const int i = x / kPrepRows, r = x % kPrepRows;
-            po.vt[(bh * D + i) * po.Wp + p0 + r] = __float2half_rn(vs[r][i]);
+        // V^T: 8 consecutive window rows of one dim per 16-byte store
+        for (int x = threadIdx.x; x < D * (kPrepRows / 8); x += blockDim.x) {
+            const int i = x / (kPrepRows / 8), r0 = (x % (kPrepRows / 8)) * 8;
+            uint4 w;
+            uint32_t *u = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const __half2 t = __floats2half2_rn(vs[r0 + 2 * e][i], vs[r0 + 2 * e + 1][i]);
+                u[e] = *reinterpret_cast<const uint32_t *>(&t);
+            }
+            *reinterpret_cast<uint4 *>(po.vt + (bh * D + i) * po.Wp + p0 + r0) = w;
         }
     } else {
         // ---- 64 query rows: rotated at W-C+c, scaled, hi/lo
@@ -170,22 +224,30 @@ prefill_prep_kernel(Geom geo, const uint16_t *__restrict__ q, const uint16_t *__
         const int R = geo.g * geo.C;
         const float qscale = 1.4426950408889634f * rsqrtf(float(D));
         const int64_t qpos0 = m.W - geo.C;
-        for (int x = threadIdx.x; x < kPrepRows * (D / 2); x += blockDim.x) {
-            const int rr = x / (D / 2), i = x % (D / 2);
+        for (int x = threadIdx.x; x < kPrepRows * NCH; x += blockDim.x) {
+            const int rr = x / NCH, i0 = (x % NCH) * 8;
             const int64_t r = r0 + rr;
-            float lo = 0.f, hi = 0.f;
+            float lo[8], hi[8];
             if (r < R) {
                 const int j = h * geo.g + int(r / geo.C), c = int(r % geo.C);
                 const uint16_t *qr = q + ((int64_t(b) * geo.Hq + j) * geo.C + c) * D;
-                const float x0 = Elem<uint16_t>::one(qr, i), x1 = Elem<uint16_t>::one(qr, i + D / 2);
-                float cs, sn;
-                rope_cs(qpos0 + c, freq[i].x, freq[i].y, cs, sn);
-                lo = (x0 * cs - x1 * sn) * qscale;
-                hi = (x1 * cs + x0 * sn) * qscale;
+                float2 cs[8];
+                const float4 *tr = reinterpret_cast<const float4 *>(tab + (qpos0 + c) * (D / 2) + i0);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 t4 = tr[e];
+                    cs[2 * e] = make_float2(t4.x, t4.y);
+                    cs[2 * e + 1] = make_float2(t4.z, t4.w);
+                }
+                rot8(*reinterpret_cast<const uint4 *>(qr + i0),
+                     *reinterpret_cast<const uint4 *>(qr + D / 2 + i0), cs, lo, hi, qscale);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) lo[e] = hi[e] = 0.f;
             }
             const int64_t qb = (bh * po.Rp + r) * D;
-            split_bf16(lo, po.qh[qb + i], po.ql[qb + i]);
-            split_bf16(hi, po.qh[qb + i + D / 2], po.ql[qb + i + D / 2]);
+            split_store(lo, po.qh + qb + i0, po.ql + qb + i0);
+            split_store(hi, po.qh + qb + D / 2 + i0, po.ql + qb + D / 2 + i0);
         }
     }
 }

@@ -271,33 +271,54 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 }
 
 // bf16 terms of the summed group query: [BH][NT][cpad][D]; rows c >= C are 0.
-template <typename T, int D>
-__global__ void qterms_kernel(Geom geo, const T *__restrict__ q, __nv_bfloat16 *__restrict__ out,
-                              int nterms, int cpad)
+// One thread per (KV head, query, 4 consecutive dims): the group sum is formed
+// once for both terms (grid.y = KV head; 32-bit index arithmetic).
+template <int D>
+__global__ void qterms_kernel(Geom geo, const uint16_t *__restrict__ q,
+                              __nv_bfloat16 *__restrict__ out, int nterms, int cpad)
 {
-    const int64_t total = int64_t(geo.B) * geo.Hkv * nterms * cpad * D;
-    for (int64_t x = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; x < total;
-         x += int64_t(gridDim.x) * blockDim.x) {
-        const int i = int(x % D);
-        const int64_t row = x / D;
-        const int c = int(row % cpad);
-        const int64_t bt = row / cpad;
-        const int term = int(bt % nterms);
-        const int64_t bh = bt / nterms;
-        const int64_t b = bh / geo.Hkv, h = bh % geo.Hkv;
-        float v = 0.f;
-        if (c < geo.C) {
-            if (nterms == geo.g) {   // the group's raw heads: exact products
-                v = Elem<T>::one(q, ((b * geo.Hq + h * geo.g + term) * geo.C + c) * D + i);
-            } else {                 // fp32 sum split into hi + lo
-                float s = 0.f;
-                for (int j = 0; j < geo.g; ++j)
-                    s += Elem<T>::one(q, ((b * geo.Hq + h * geo.g + j) * geo.C + c) * D + i);
-                const float hi = __bfloat162float(__float2bfloat16_rn(s));
-                v = term == 0 ? hi : s - hi;
+    constexpr int D4 = D / 4;
+    const int x = blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= cpad * D4) return;
+    const int c = x / D4, i0 = (x % D4) * 4;
+    const int bh = blockIdx.y;
+    const int b = bh / geo.Hkv, h = bh % geo.Hkv;
+    float v[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    if (c < geo.C) {
+        if (nterms == geo.g) {   // the group's raw heads: exact products
+            for (int term = 0; term < nterms; ++term) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(
+                    q + ((int64_t(b) * geo.Hq + h * geo.g + term) * geo.C + c) * D + i0);
+                v[term][0] = bf16lo(w.x);
+                v[term][1] = bf16hi(w.x);
+                v[term][2] = bf16lo(w.y);
+                v[term][3] = bf16hi(w.y);
+            }
+        } else {                 // fp32 sum split into hi + lo
+            float sum[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int j = 0; j < geo.g; ++j) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(
+                    q + ((int64_t(b) * geo.Hq + h * geo.g + j) * geo.C + c) * D + i0);
+                sum[0] += bf16lo(w.x);
+                sum[1] += bf16hi(w.x);
+                sum[2] += bf16lo(w.y);
+                sum[3] += bf16hi(w.y);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float hi = __bfloat162float(__float2bfloat16_rn(sum[e]));
+                v[0][e] = hi;
+                v[1][e] = sum[e] - hi;
             }
         }
-        out[x] = __float2bfloat16_rn(v);
+    }
+    for (int term = 0; term < nterms; ++term) {
+        __nv_bfloat162 lo2 = __floats2bfloat162_rn(v[term][0], v[term][1]);
+        __nv_bfloat162 hi2 = __floats2bfloat162_rn(v[term][2], v[term][3]);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t *>(&lo2);
+        w.y = *reinterpret_cast<const uint32_t *>(&hi2);
+        *reinterpret_cast<uint2 *>(out + ((int64_t(bh) * nterms + term) * cpad + c) * D + i0) = w;
     }
 }
 
@@ -358,14 +379,13 @@ cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, fl
     ta.nterms = tc_terms(geo);
     if (ta.items == 0) return cudaSuccess;
     __nv_bfloat16 *terms = static_cast<__nv_bfloat16 *>(scratch);
-    const int64_t n = int64_t(geo.B) * geo.Hkv * ta.nterms * ta.cpad * geo.d;
-    const int blocks = int((n + 255) / 256 < 8192 ? (n + 255) / 256 : 8192);
+    const dim3 qgrid(unsigned((ta.cpad * (geo.d / 4) + 255) / 256), unsigned(geo.B * geo.Hkv));
     if (geo.d == 128)
-        qterms_kernel<uint16_t, 128><<<blocks, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q),
-                                                             terms, ta.nterms, ta.cpad);
+        qterms_kernel<128><<<qgrid, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q), terms,
+                                                  ta.nterms, ta.cpad);
     else
-        qterms_kernel<uint16_t, 64><<<blocks, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q),
-                                                            terms, ta.nterms, ta.cpad);
+        qterms_kernel<64><<<qgrid, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q), terms,
+                                                 ta.nterms, ta.cpad);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     CUtensorMap kmap, qmap;
