@@ -329,12 +329,24 @@ REATT_API int reatt_merge_partials(const reatt_dims *dims, int32_t n_parts,
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents; what must start at zero is cleared inside each call.  Calls
  *     that overlap on the GPU race: order them on one stream.
- *   - A bounded-wait timeout is recorded in the shared array's status word,
- *     which this call does not expose.
+ *   - A bounded-wait timeout is recorded in the shared array's status word
+ *     (offset 0), like any workspace's: pass reatt_fixed_scratch_address()'s
+ *     result to reatt_workspace_status() to read and clear it.
  */
 REATT_API int reatt_step_fixed_scratch(const reatt_dims *dims, const void *q, const void *k_cache,
                                        const void *v_cache, const void *k_cur, const void *v_cur,
                                        int32_t *sel_out, float *out, reatt_stream stream);
+
+/*
+ * Device address of the fixed scratch that reatt_step_fixed_scratch uses, on
+ * the current device (looked up on every call, like the step does; the first
+ * call on a device loads the library's device globals there).  It is meant
+ * for reatt_workspace_status() and reatt_selftest_bounded_wait(); the array's
+ * other contents belong to the library and change with every fixed-scratch
+ * step.  *ws_out is set only on REATT_OK.  EINVAL for a null ws_out, ECUDA if
+ * the lookup fails.
+ */
+REATT_API int reatt_fixed_scratch_address(void **ws_out);
 
 #ifdef __cplusplus
 }

@@ -124,6 +124,7 @@ def test_null_dims_and_outputs(R):
     assert R.lib.reatt_workspace_bytes(ctypes.byref(dims(R)), None) == 1
     st = ctypes.c_int()
     assert R.lib.reatt_workspace_status(None, ctypes.byref(st), None) == 1
+    assert R.lib.reatt_fixed_scratch_address(None) == 1
 
 
 def test_null_and_misaligned_pointers(R):

@@ -59,3 +59,30 @@ def test_fixed_scratch_rejects_oversized_work(R):
     rc = R.lib.reatt_step_fixed_scratch(ctypes.byref(d), fake, fake, fake, fake, fake, None, fake,
                                         None)
     assert rc == R.EUNSUPPORTED
+
+
+def test_fixed_scratch_status_word_reports_a_timeout(R):
+    """A bounded-wait timeout in the fixed array is visible to the caller
+    through its address, the read clears it, and the next step is normal."""
+    torch.cuda.init()
+    ws = R.reatt_fixed_scratch_address()
+    assert ws % 256 == 0
+    assert R.reatt_fixed_scratch_address() == ws
+    assert R.reatt_workspace_status(ws) == R.OK
+    R.reatt_selftest_bounded_wait(ws, 20_000_000)        # 20 ms
+    torch.cuda.synchronize()
+    assert R.reatt_workspace_status(ws) == R.ETIMEOUT
+    assert R.reatt_workspace_status(ws) == R.OK          # read clears it
+    w = CASES[0]
+    x = {n: t.cuda() for n, t in wl.make_inputs(w).items() if n != "needles"}
+    d = R.dims_of(w)
+    b = R.alloc_outputs(d)
+    R.reatt_step(d, x["q"], x["k_cache"], x["v_cache"], x["k_cur"], x["v_cur"], b["sel"],
+                 b["out"], b["ws"])
+    sel = torch.empty_like(b["sel"])
+    out = torch.empty_like(b["out"])
+    R.reatt_step_fixed_scratch(d, x["q"], x["k_cache"], x["v_cache"], x["k_cur"], x["v_cur"],
+                               sel, out)
+    torch.cuda.synchronize()
+    assert R.reatt_workspace_status(ws) == R.OK
+    assert torch.equal(sel, b["sel"])

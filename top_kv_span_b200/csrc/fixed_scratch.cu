@@ -47,3 +47,9 @@ extern "C" REATT_API int reatt_step_fixed_scratch(const reatt_dims *dims, const 
     if (sc != REATT_OK) return sc;
     return reatt_step(dims, q, k_cache, v_cache, k_cur, v_cur, sel_out, out, ws, stream);
 }
+
+extern "C" REATT_API int reatt_fixed_scratch_address(void **ws_out)
+{
+    if (!ws_out) return REATT_EINVAL;
+    return scratch_on_current_device(ws_out);
+}

@@ -21,7 +21,7 @@ F32, BF16 = 0, 1
 EXPORTS = ["reatt_status_string", "reatt_num_spans", "reatt_window_max", "reatt_workspace_bytes",
            "reatt_workspace_status", "reatt_score_spans", "reatt_topk", "reatt_gather_rope",
            "reatt_attend", "reatt_step", "reatt_append_kv", "reatt_selftest_bounded_wait",
-           "reatt_step_fixed_scratch", "reatt_shard_plan", "reatt_shard_workspace_bytes",
+           "reatt_step_fixed_scratch", "reatt_fixed_scratch_address", "reatt_shard_plan", "reatt_shard_workspace_bytes",
            "reatt_shard_candidates", "reatt_shard_select", "reatt_shard_attend",
            "reatt_merge_partials"]
 
@@ -216,6 +216,14 @@ def reatt_step_fixed_scratch(dims, q, k_cache, v_cache, k_cur, v_cur, sel_out, o
     if check:
         _check(rc, "reatt_step_fixed_scratch")
     return rc
+
+
+def reatt_fixed_scratch_address() -> int:
+    """Device address of the fixed scratch on the current device, for
+    reatt_workspace_status (its status word) and the bounded-wait selftest."""
+    p = ctypes.c_void_p()
+    _check(lib.reatt_fixed_scratch_address(ctypes.byref(p)), "reatt_fixed_scratch_address")
+    return int(p.value)
 
 
 def reatt_shard_plan(dims, n):
