@@ -10,11 +10,13 @@ outside each step's CUDA-event interval.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl ours|reference] [--extra NAMES] [--loops NAMES]
+                  [--prefill-loop NAME]
 
 At N=1 the same line also carries `per_workload` (the other workloads: the
 tiny fp32 decode, the 1M x 4 and 4M decodes, the 2048-query prefill chunk),
 each with its own timings, roofline and a parity sample, and `decode_loop`
-(a graph-replayed decoding loop with its appends).  Parity comes from the
+(a graph-replayed decoding loop with its appends) and `prefill_loop` (a
+128K-token prompt prefilled in the pages' chunks, each appended).  Parity comes from the
 CPU leg, which runs the oracle on a bounded sample (KV head 0 of sequence 0)
 and compares the GPU's selection (swap count) and outputs (max-abs) on it.
 
@@ -519,6 +521,54 @@ def decode_loop(w, dev, timer, n_steps=16, reps=10):
             "note": "median over replays; one L2 flush before each loop of steps"}
 
 
+def prefill_loop(w, dev, timer, prompt=131072, chunk=512, reps=3):
+    """NEXT step of a prefill as the pages run it: a first chunk of G+L
+    tokens over an empty cache, then chunks of `chunk` tokens (chunk_size=512
+    in the OpenReview discussion's NIAH settings), each attending over the
+    cache built so far (span selection on its middle) and then appended in
+    place (caches with T_cap = prompt rows).  Launched eagerly; L2 flushed
+    before each prompt, not between its chunks."""
+    import torch
+    from top_kv_span_b200 import reatt as R
+
+    first = w.G + w.L
+    n = max(0, (prompt - first) // chunk)
+    sizes = [first] + [chunk] * n
+    P = sum(sizes)
+    gen = torch.Generator(device=dev).manual_seed(w.seed + 91)
+    rnd = lambda shp: torch.randn(shp, generator=gen, device=dev).to(w.torch_dtype)
+    # per-chunk contiguous operands: [B, Hq, c, d] queries, [B, Hkv, c, d] K/V
+    qs = [rnd((w.B, w.Hq, c, w.d)) for c in sizes]
+    kn = [rnd((w.B, w.Hkv, c, w.d)) for c in sizes]
+    vn = [rnd((w.B, w.Hkv, c, w.d)) for c in sizes]
+    kc = torch.zeros((w.B, w.Hkv, P, w.d), dtype=w.torch_dtype, device=dev)
+    vc = torch.zeros_like(kc)
+    dims, t = [], 0
+    for c in sizes:
+        dims.append(R.dims_of(w, T=t, C=c, T_cap=P))
+        t += c
+    ws = torch.zeros(max(R.reatt_workspace_bytes(dd) for dd in dims), dtype=torch.uint8,
+                     device=dev)
+    outs = {c: torch.empty((w.B, w.Hq, c, w.d), dtype=torch.float32, device=dev)
+            for c in set(sizes)}
+    sel = torch.empty((w.B, w.Hkv, w.k), dtype=torch.int32, device=dev)
+    st = timer.stream
+
+    def one_prompt(i=0):
+        for j, c in enumerate(sizes):
+            R.reatt_step(dims[j], qs[j], kc, vc, kn[j], vn[j], sel, outs[c], ws, stream=st)
+            R.reatt_append_kv(dims[j], kc, vc, kn[j], vn[j], stream=st)
+
+    ms = timer.run(one_prompt, reps, warmup=1)
+    assert R.reatt_workspace_status(ws, st) == R.OK
+    med = statistics.median(ms)
+    return {"workload": w.name, "prompt_tokens": P, "first_chunk": first, "chunk": chunk,
+            "chunks": len(sizes), "ms_per_prompt": round(med, 3),
+            "tokens_per_s": round(P / (med * 1e-3), 1),
+            "us_per_chunk": round(med * 1e3 / len(sizes), 2),
+            "note": "eager launches; median over prompts; one L2 flush before each prompt"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -565,6 +615,9 @@ def run_ours(args):
         torch.cuda.empty_cache()
         result["decode_loop"] = {name: decode_loop(wl.WORKLOADS[name], dev, timer)
                                  for name in args.loops.split(",") if name}
+    if world == 1 and args.prefill_loop:
+        torch.cuda.empty_cache()
+        result["prefill_loop"] = prefill_loop(wl.WORKLOADS[args.prefill_loop], dev, timer)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -753,6 +806,9 @@ def main():
                          "'' for none")
     ap.add_argument("--loops", default="tiny_f32_4k,llama3_8b_128k",
                     help="workloads whose graph-replayed decoding loop is timed (N=1 only)")
+    ap.add_argument("--prefill-loop", default="llama3_8b_128k",
+                    help="workload whose heads time a chunked 128K-token prefill "
+                         "(first chunk G+L, then 512-token chunks with appends); '' skips it")
     ap.add_argument("--launch-check", action="store_true",
                     help="multi-rank plumbing only, on CPU ranks (gloo), no GPU work")
     args = ap.parse_args()

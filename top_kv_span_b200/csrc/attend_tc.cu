@@ -14,20 +14,24 @@
 // (hi/lo), the rotated window keys (hi/lo) and the window values transposed
 // (fp16), from the un-rotated cache through the selection (the window is
 // never materialised in fp32).  attend_prefill_tc_kernel then runs, per
-// 128-row query block:
-//   warp 0   TMA producer: the query block once, then 64-key tiles of K (hi,
-//            lo) and V^T in a 2-stage ring (128B swizzle, no multicast)
+// 128-row query block (TMEM lanes = query rows):
+//   warp 0   TMA producer: 64-key tiles of K (hi, lo) into a 4-stage ring
+//            and V^T into a 3-stage ring, each issued as soon as its stage
+//            is free (128B swizzle, no multicast)
 //   warp 1   TMEM allocation; one thread issues, whichever is ready, S(j)
-//            into one of two TMEM S buffers and O += P(j).V(j) into the TMEM
-//            O accumulator (S never waits behind a P.V)
+//            into one of two TMEM S tiles and O += P(j).V(j) into the TMEM
+//            O accumulator (S never waits behind a P.V).  Both products read
+//            their A operand (the query terms, P) from TMEM, so only K and
+//            V^T are read from shared memory
 //   warps 2-9 softmax: two warps per TMEM lane group, one per 32-column half
-//            of the S tile; a thread owns one query row's half: it reads its
+//            of the S tile; first each stores its rows' query term (hi or
+//            lo) into TMEM.  A thread owns one query row's half: it reads its
 //            32 S values from TMEM, masks (causal, window end), trades its
 //            half-row max with the partner warp (a named barrier per pair),
 //            keeps a running reference max that moves (and rescales its half
 //            of O in TMEM) only when the row max grows by more than 2^8,
-//            writes its half of P in the swizzled operand layout into one of
-//            two P buffers, and finally divides its half of O by the row sum.
+//            stores its half of P as fp16 pairs into one of two TMEM P tiles,
+//            and finally divides its half of O by the row sum.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -255,28 +259,33 @@ prefill_prep_kernel(Geom geo, const uint16_t *__restrict__ q, const uint16_t *__
 struct FaArgs {
     float *out;
     const int32_t *sel;
+    const __nv_bfloat16 *qh, *ql;   // [BH][Rp][D] query operand terms
     int Rp, Wp;
 };
 
-// Shared-memory plan (1024-byte aligned): Qh | Ql | K stage 0,1 (hi | lo) |
-// V^T stage 0,1 | Ph | Pl | barriers.
+constexpr int kKStages = 4;   // K tiles (hi | lo) in flight
+constexpr int kVStages = 3;   // V^T tiles in flight
+
+// Shared-memory plan (1024-byte aligned): K stages (hi | lo) | V^T stages |
+// barriers.  The query terms and P live in TMEM.
 template <int D>
 struct FaSmem {
     static constexpr int NBOX = D / 64;
-    static constexpr int kQ = NBOX * kQRows * 128;       // one of Qh / Ql
     static constexpr int kK = NBOX * kKeyTile * 128;     // one of Kh / Kl
     static constexpr int kV = D * kKeyTile * 2;          // V^T tile: D rows x 64 keys
-    static constexpr int kP = kQRows * kKeyTile * 2;     // one of Ph / Pl
-    static constexpr int oQh = 0, oQl = kQ, oK = 2 * kQ, oV = oK + 4 * kK, oP = oV + 2 * kV,
-                         oBar = oP + 2 * kP;
+    static constexpr int oK = 0, oV = kKStages * 2 * kK, oBar = oV + kVStages * kV;
     static constexpr size_t kBytes = size_t(oBar) + 32 * 8 + 1024;
 };
 
+// TMEM columns of one CTA (128 lanes = the query rows): two S tiles, the O
+// accumulator, the query terms (A operand of S: lane = row, two bf16 of the
+// head width per column) and two P tiles (A operand of P.V, two fp16 keys
+// per column).
+constexpr uint32_t kSCol = 0, kOCol = 128, kQCol = 256, kPCol = 384, kTmemCols = 512;
+
 template <int D>
 __global__ void __launch_bounds__(kFaThreads, 1)
-attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
-                         const __grid_constant__ CUtensorMap qlmap,
-                         const __grid_constant__ CUtensorMap khmap,
+attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
                          const __grid_constant__ CUtensorMap klmap,
                          const __grid_constant__ CUtensorMap vtmap, Geom geo, FaArgs fa, void *ws)
 {
@@ -284,26 +293,31 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
     constexpr int NBOX = Sm::NBOX;
     constexpr int KS = D / 16;                 // k-steps of S over the head width
     constexpr int PS = kKeyTile / 16;          // k-steps of P.V over a key tile
-    constexpr uint32_t kTmemCols = 256;        // S buffers at 0 and 64, O at 128
+    static_assert(kOCol + D <= kQCol && kQCol + D <= kPCol && kPCol + 2 * kKeyTile / 2 <= kTmemCols,
+                  "TMEM plan");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Sm::oBar);
-    uint64_t *qfull = bars, *kfull = bars + 1, *kempty = bars + 3, *vfull = bars + 5,
-             *vempty = bars + 7, *sfull = bars + 9, *sempty = bars + 11, *pfull = bars + 13,
-             *pvdone = bars + 15, *done = bars + 17;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 18);
+    uint64_t *qfull = bars, *kfull = bars + 1, *kempty = kfull + kKStages,
+             *vfull = kempty + kKStages, *vempty = vfull + kVStages, *sfull = vempty + kVStages,
+             *sempty = sfull + 2, *pfull = sempty + 2, *pvdone = pfull + 2, *done = pvdone + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         abort_flag = 0;
-        mbar_init(qfull, 1);
-        for (int s = 0; s < 2; ++s) {
+        mbar_init(qfull, kFaSoftWarps);   // query terms stored in TMEM (one arrival per softmax warp)
+        for (int s = 0; s < kKStages; ++s) {
             mbar_init(&kfull[s], 1);
             mbar_init(&kempty[s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
             mbar_init(&vfull[s], 1);
             mbar_init(&vempty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&sfull[s], 1);
             mbar_init(&sempty[s], kFaSoftWarps);
             mbar_init(&pfull[s], kFaSoftWarps);   // P buffer s written (one arrival per softmax warp)
@@ -344,47 +358,58 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
+        // K and V^T tiles go through separate rings and are issued, in
+        // tile order within each ring, as soon as a stage is free (K first:
+        // the next S needs it before the next P.V needs its V).
         if (lane == 0) {
             bool ok = true;
-            const int qy = int(bh * fa.Rp + r0);
-            mbar_arrive_expect_tx(qfull, 2 * Sm::kQ);
-            for (int bx = 0; bx < NBOX; ++bx) {
-                tma_load_2d(smem + Sm::oQh + bx * kQRows * 128, &qhmap, 64 * bx, qy, qfull);
-                tma_load_2d(smem + Sm::oQl + bx * kQRows * 128, &qlmap, 64 * bx, qy, qfull);
-            }
-            for (int j = 0; ok && j < nt; ++j) {
-                const int s = j & 1;
-                if (j >= 2 && (aborted() || !mbar_wait_bounded(&kempty[s], ((j >> 1) - 1) & 1, kWaitLimitNs))) {
+            int jk = 0, jv = 0;
+            uint64_t t_last = global_ns();
+            while (ok && (jk < nt || jv < nt)) {
+                bool progressed = false;
+                if (jk < nt) {
+                    const int s = jk % kKStages, u = jk / kKStages;
+                    if (u == 0 || mbar_test(&kempty[s], (u - 1) & 1)) {
+                        const int ky = int(bh * fa.Wp + int64_t(jk) * kKeyTile);
+                        uint8_t *kst = smem + Sm::oK + s * 2 * Sm::kK;
+                        mbar_arrive_expect_tx(&kfull[s], 2 * Sm::kK);
+                        for (int bx = 0; bx < NBOX; ++bx) {
+                            tma_load_2d(kst + bx * kKeyTile * 128, &khmap, 64 * bx, ky, &kfull[s]);
+                            tma_load_2d(kst + Sm::kK + bx * kKeyTile * 128, &klmap, 64 * bx, ky, &kfull[s]);
+                        }
+                        ++jk;
+                        progressed = true;
+                    }
+                }
+                if (jv < jk) {
+                    const int s = jv % kVStages, u = jv / kVStages;
+                    if (u == 0 || mbar_test(&vempty[s], (u - 1) & 1)) {
+                        mbar_arrive_expect_tx(&vfull[s], Sm::kV);
+                        tma_load_2d(smem + Sm::oV + s * Sm::kV, &vtmap, jv * kKeyTile, int(bh * D), &vfull[s]);
+                        ++jv;
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    t_last = global_ns();
+                } else if (aborted() || global_ns() - t_last > kWaitLimitNs) {
                     fail();
                     ok = false;
-                    break;
+                } else {
+                    __nanosleep(64);
                 }
-                const int ky = int(bh * fa.Wp + int64_t(j) * kKeyTile);
-                uint8_t *kst = smem + Sm::oK + s * 2 * Sm::kK;
-                mbar_arrive_expect_tx(&kfull[s], 2 * Sm::kK);
-                for (int bx = 0; bx < NBOX; ++bx) {
-                    tma_load_2d(kst + bx * kKeyTile * 128, &khmap, 64 * bx, ky, &kfull[s]);
-                    tma_load_2d(kst + Sm::kK + bx * kKeyTile * 128, &klmap, 64 * bx, ky, &kfull[s]);
-                }
-                if (j >= 2 && (aborted() || !mbar_wait_bounded(&vempty[s], ((j >> 1) - 1) & 1, kWaitLimitNs))) {
-                    fail();
-                    ok = false;
-                    break;
-                }
-                mbar_arrive_expect_tx(&vfull[s], Sm::kV);
-                tma_load_2d(smem + Sm::oV + s * Sm::kV, &vtmap, j * kKeyTile, int(bh * D), &vfull[s]);
             }
-            // drain the loads in flight
-            if (!mbar_wait_bounded(qfull, 0, kWaitLimitNs)) fail();
-            for (int j = nt - 2 < 0 ? 0 : nt - 2; j < nt; ++j) {
-                if (!mbar_wait_bounded(&kfull[j & 1], (j >> 1) & 1, kWaitLimitNs)) fail();
-                if (!mbar_wait_bounded(&vfull[j & 1], (j >> 1) & 1, kWaitLimitNs)) fail();
-            }
+            // drain the loads in flight (the last fill of each stage)
+            for (int j = jk - kKStages < 0 ? 0 : jk - kKStages; j < jk; ++j)
+                if (!mbar_wait_bounded(&kfull[j % kKStages], (j / kKStages) & 1, kWaitLimitNs)) fail();
+            for (int j = jv - kVStages < 0 ? 0 : jv - kVStages; j < jv; ++j)
+                if (!mbar_wait_bounded(&vfull[j % kVStages], (j / kVStages) & 1, kWaitLimitNs)) fail();
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(kQRows, kKeyTile), id_o = idesc_f16(kQRows, D);
+            const uint32_t t_qh = tmem_base + kQCol, t_ql = t_qh + uint32_t(D / 2);
             bool ok = !aborted() && mbar_wait_bounded(qfull, 0, kWaitLimitNs);
             if (!ok) fail();
             tc_fence_after();
@@ -396,42 +421,43 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
             uint64_t t_last = global_ns();
             while (ok && jp < nt) {
                 bool progressed = false;
-                if (js < nt && mbar_test(&kfull[js & 1], (js >> 1) & 1) &&
+                if (js < nt && mbar_test(&kfull[js % kKStages], (js / kKStages) & 1) &&
                     (js < 2 || mbar_test(&sempty[js & 1], ((js >> 1) - 1) & 1))) {
-                    const int s = js & 1;   // S(js) = Q.K(js)^T (three hi/lo products)
+                    // S(js) = Q.K(js)^T (three hi/lo products; Q from TMEM)
+                    const int s = js & 1, ks_ = js % kKStages;
                     tc_fence_after();
-                    const uint8_t *kst = smem + Sm::oK + s * 2 * Sm::kK;
-                    const uint32_t d_s = tmem_base + uint32_t(s * kKeyTile);
+                    const uint8_t *kst = smem + Sm::oK + ks_ * 2 * Sm::kK;
+                    const uint32_t d_s = tmem_base + kSCol + uint32_t(s * kKeyTile);
 #pragma unroll
                     for (int ks = 0; ks < KS; ++ks) {
                         const int bx = ks / 4, kin = ks % 4;
-                        const uint64_t qh = sw128_desc(smem + Sm::oQh + bx * kQRows * 128) + uint64_t(kin * 2);
-                        const uint64_t ql = sw128_desc(smem + Sm::oQl + bx * kQRows * 128) + uint64_t(kin * 2);
                         const uint64_t kh = sw128_desc(kst + bx * kKeyTile * 128) + uint64_t(kin * 2);
                         const uint64_t kl = sw128_desc(kst + Sm::kK + bx * kKeyTile * 128) + uint64_t(kin * 2);
-                        tc_mma(d_s, qh, kh, id_s, ks > 0 ? 1u : 0u);
-                        tc_mma(d_s, qh, kl, id_s, 1u);
-                        tc_mma(d_s, ql, kh, id_s, 1u);
+                        const uint32_t qh = t_qh + uint32_t(ks * 8), ql = t_ql + uint32_t(ks * 8);
+                        tc_mma_ts(d_s, qh, kh, id_s, ks > 0 ? 1u : 0u);
+                        tc_mma_ts(d_s, qh, kl, id_s, 1u);
+                        tc_mma_ts(d_s, ql, kh, id_s, 1u);
                     }
                     tc_commit(&sfull[s]);
-                    tc_commit(&kempty[s]);
+                    tc_commit(&kempty[ks_]);
                     ++js;
                     progressed = true;
                 }
                 if (jp < js && mbar_test(&pfull[jp & 1], (jp >> 1) & 1) &&
-                    mbar_test(&vfull[jp & 1], (jp >> 1) & 1)) {
-                    const int s = jp & 1;   // O += P(jp).V(jp)
+                    mbar_test(&vfull[jp % kVStages], (jp / kVStages) & 1)) {
+                    // O += P(jp).V(jp) (P from TMEM)
+                    const int s = jp & 1, vs_ = jp % kVStages;
                     tc_fence_after();
-                    const uint32_t d_o = tmem_base + 128u;
-                    const uint8_t *vst = smem + Sm::oV + s * Sm::kV;
+                    const uint32_t d_o = tmem_base + kOCol;
+                    const uint32_t t_p = tmem_base + kPCol + uint32_t(s * (kKeyTile / 2));
+                    const uint8_t *vst = smem + Sm::oV + vs_ * Sm::kV;
 #pragma unroll
                     for (int ks = 0; ks < PS; ++ks) {
-                        const uint64_t pd = sw128_desc(smem + Sm::oP + s * Sm::kP) + uint64_t(ks * 2);
                         const uint64_t vd = sw128_desc(vst) + uint64_t(ks * 2);
-                        tc_mma(d_o, pd, vd, id_o, (jp > 0 || ks > 0) ? 1u : 0u);
+                        tc_mma_ts(d_o, t_p + uint32_t(ks * 8), vd, id_o, (jp > 0 || ks > 0) ? 1u : 0u);
                     }
                     tc_commit(&pvdone[s]);
-                    tc_commit(&vempty[s]);
+                    tc_commit(&vempty[vs_]);
                     ++jp;
                     progressed = true;
                 }
@@ -467,8 +493,31 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
         auto pair_sync = [&] { named_sync(1 + quad, 64); };
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
-        uint8_t *pbuf = smem + Sm::oP;
         constexpr int HC = kKeyTile / 2;         // columns per warp
+        {
+            // this row's query term (half 0: hi, half 1: lo) into TMEM, the
+            // A operand of S; rows >= R are zero in the prep's buffer
+            const __nv_bfloat16 *src = (half ? fa.ql : fa.qh) + (bh * fa.Rp + r0 + row) * D;
+            const uint32_t tq = lane_base + kQCol + uint32_t(half * (D / 2));
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+                float w[32];
+                const uint4 *s4 = reinterpret_cast<const uint4 *>(src + c * 64);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 v = s4[i];
+                    w[4 * i] = __uint_as_float(v.x);
+                    w[4 * i + 1] = __uint_as_float(v.y);
+                    w[4 * i + 2] = __uint_as_float(v.z);
+                    w[4 * i + 3] = __uint_as_float(v.w);
+                }
+                tmem_st32(tq + uint32_t(c * 32), w);
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(qfull);
+        }
         for (int j = 0; j < nt; ++j) {
             const int s = j & 1;
             if (ok) {
@@ -539,38 +588,32 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
 #pragma unroll
                 for (int cb = 0; cb < D / 64; ++cb) {
                     float o[32];
-                    const uint32_t ta = lane_base + 128u + uint32_t(half * (D / 2) + cb * 32);
+                    const uint32_t ta = lane_base + kOCol + uint32_t(half * (D / 2) + cb * 32);
                     tmem_ld32(ta, o);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] *= fac;
                     tmem_st32(ta, o);
                 }
             }
-            // P = exp2(S - m_ref) <= 2^8 as fp16 (11-bit significand), 128B-
-            // swizzled K-major rows of buffer j&1; this warp writes chunks
-            // [4*half, 4*half + 4) of the row
+            // P = exp2(S - m_ref) <= 2^8 as fp16 (11-bit significand) into
+            // this row's lane of TMEM P buffer j&1: keys [32*half, 32*half+32)
+            // as 16 columns of fp16 pairs (the A operand of P.V)
             const bool any_key = m_ref != -INFINITY;
-            uint8_t *pw = pbuf + s * Sm::kP + row * 128;
             float rs = 0.f;
+            float pw[HC / 2];
 #pragma unroll
-            for (int c = 0; c < HC / 8; ++c) {
-                uint32_t hw[4];
-#pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    // masked keys are -inf: ex2 gives 0; a row with no key
-                    // seen yet (m_ref = -inf) has only masked keys
-                    const float p0 = any_key ? ex2_approx(sv[c * 8 + e] - m_ref) : 0.f;
-                    const float p1 = any_key ? ex2_approx(sv[c * 8 + e + 1] - m_ref) : 0.f;
-                    rs += p0 + p1;
-                    const __half2 hv = __floats2half2_rn(p0, p1);
-                    hw[e / 2] = *reinterpret_cast<const uint32_t *>(&hv);
-                }
-                const int ch = half * (HC / 8) + c;
-                *reinterpret_cast<uint4 *>(pw + (ch ^ (row & 7)) * 16) =
-                    make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            for (int e = 0; e < HC; e += 2) {
+                // masked keys are -inf: ex2 gives 0; a row with no key seen
+                // yet (m_ref = -inf) has only masked keys
+                const float p0 = any_key ? ex2_approx(sv[e] - m_ref) : 0.f;
+                const float p1 = any_key ? ex2_approx(sv[e + 1] - m_ref) : 0.f;
+                rs += p0 + p1;
+                const __half2 hv = __floats2half2_rn(p0, p1);
+                pw[e / 2] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&hv));
             }
+            tmem_st16(lane_base + kPCol + uint32_t(s * (kKeyTile / 2) + half * (HC / 2)), pw);
             l += rs;
-            fence_proxy_async_smem();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&pfull[s]);
         }
@@ -593,7 +636,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap qhmap,
 #pragma unroll
                 for (int cb = 0; cb < D / 64; ++cb) {
                     float o[32];
-                    tmem_ld32(lane_base + 128u + uint32_t(half * (D / 2) + cb * 32), o);
+                    tmem_ld32(lane_base + kOCol + uint32_t(half * (D / 2) + cb * 32), o);
                     if (live) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
@@ -709,14 +752,15 @@ cudaError_t launch_attend_prefill_tc(const Geom &geo, const void *q, const void 
                        sel, tab, po);
     if (e != cudaSuccess) return e;
     const uint64_t BHu = BH;
-    CUtensorMap qh, ql, kh, kl, vt;
-    if (!map2d(&qh, po.qh, BHu * pp.Rp, geo.d, kQRows) || !map2d(&ql, po.ql, BHu * pp.Rp, geo.d, kQRows) ||
-        !map2d(&kh, po.kh, BHu * pp.Wp, geo.d, kKeyTile) || !map2d(&kl, po.kl, BHu * pp.Wp, geo.d, kKeyTile) ||
+    CUtensorMap kh, kl, vt;
+    if (!map2d(&kh, po.kh, BHu * pp.Wp, geo.d, kKeyTile) || !map2d(&kl, po.kl, BHu * pp.Wp, geo.d, kKeyTile) ||
         !map2d(&vt, po.vt, BHu * geo.d, pp.Wp, uint32_t(geo.d)))
         return cudaErrorInvalidValue;
     FaArgs fa;
     fa.out = out;
     fa.sel = sel;
+    fa.qh = po.qh;
+    fa.ql = po.ql;
     fa.Rp = pp.Rp;
     fa.Wp = pp.Wp;
     dim3 grid(unsigned(pp.Rp / kQRows), BH);
@@ -724,12 +768,12 @@ cudaError_t launch_attend_prefill_tc(const Geom &geo, const void *q, const void 
         auto kern = attend_prefill_tc_kernel<128>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(FaSmem<128>::kBytes));
         if (e != cudaSuccess) return e;
-        e = launch_pdl(kern, grid, dim3(kFaThreads), FaSmem<128>::kBytes, st, qh, ql, kh, kl, vt, geo, fa, ws);
+        e = launch_pdl(kern, grid, dim3(kFaThreads), FaSmem<128>::kBytes, st, kh, kl, vt, geo, fa, ws);
     } else {
         auto kern = attend_prefill_tc_kernel<64>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(FaSmem<64>::kBytes));
         if (e != cudaSuccess) return e;
-        e = launch_pdl(kern, grid, dim3(kFaThreads), FaSmem<64>::kBytes, st, qh, ql, kh, kl, vt, geo, fa, ws);
+        e = launch_pdl(kern, grid, dim3(kFaThreads), FaSmem<64>::kBytes, st, kh, kl, vt, geo, fa, ws);
     }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
