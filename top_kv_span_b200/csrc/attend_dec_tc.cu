@@ -340,7 +340,7 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
             // S(js) as soon as tile js is converted (and its S buffer read),
             // P(jp).V(jp) as soon as P(jp) is written: whichever is ready.
             int js = 0, jp = 0;
-            uint64_t t_last = global_ns();
+            IdleWatch watch;
             while (qok && jp < nt) {
                 bool progressed = false;
                 if (js < nt && mbar_test(kopfull, uint32_t(js) & 1u) &&
@@ -381,8 +381,8 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                     progressed = true;
                 }
                 if (progressed) {
-                    t_last = global_ns();
-                } else if (aborted() || global_ns() - t_last > kWaitLimitNs) {
+                    watch.progress();
+                } else if (aborted() || watch.expired(kWaitLimitNs)) {
                     fail();
                     break;
                 } else {

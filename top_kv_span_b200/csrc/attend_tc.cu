@@ -18,11 +18,13 @@
 //   warp 0   TMA producer: 64-key tiles of K (hi, lo) into a 4-stage ring
 //            and V^T into a 3-stage ring, each issued as soon as its stage
 //            is free (128B swizzle, no multicast)
-//   warp 1   TMEM allocation; one thread issues, whichever is ready, S(j)
-//            into one of two TMEM S tiles and O += P(j).V(j) into the TMEM
-//            O accumulator (S never waits behind a P.V).  Both products read
-//            their A operand (the query terms, P) from TMEM, so only K and
-//            V^T are read from shared memory
+//   warp 1   TMEM allocation; one thread issues S(j) into one of two TMEM
+//            S tiles as soon as K(j) has landed and the tile is free
+//   warp 10  one thread issues O += P(j).V(j) into the TMEM O accumulator
+//            as soon as P(j) is written (a thread of its own: tcgen05.mma
+//            issue stalls while the pipe is full, and a P.V must not wait
+//            behind an S).  Both products read their A operand (the query
+//            terms, P) from TMEM, so only K and V^T come from shared memory
 //   warps 2-9 softmax: two warps per TMEM lane group, one per 32-column half
 //            of the S tile; first each stores its rows' query term (hi or
 //            lo) into TMEM.  A thread owns one query row's half: it reads its
@@ -48,8 +50,9 @@ namespace {
 
 using namespace tc;
 
-constexpr int kFaSoftWarps = 8;          // two per TMEM lane group
-constexpr int kFaThreads = (2 + kFaSoftWarps) * 32;
+constexpr int kFaSoftWarps = 8;          // two per TMEM lane group (warps 2..9)
+constexpr int kFaPvWarp = 2 + kFaSoftWarps;   // issues the P.V products
+constexpr int kFaThreads = (3 + kFaSoftWarps) * 32;
 constexpr int kQRows = 128;   // query rows per CTA (TMEM lanes)
 constexpr int kKeyTile = 64;  // keys per S tile (S columns)
 constexpr float kRescaleLog2 = 8.f;
@@ -302,7 +305,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
     uint64_t *qfull = bars, *kfull = bars + 1, *kempty = kfull + kKStages,
              *vfull = kempty + kKStages, *vempty = vfull + kVStages, *sfull = vempty + kVStages,
              *sempty = sfull + 2, *pfull = sempty + 2, *pvdone = pfull + 2, *done = pvdone + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 2);
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -323,7 +326,8 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
             mbar_init(&pfull[s], kFaSoftWarps);   // P buffer s written (one arrival per softmax warp)
             mbar_init(&pvdone[s], 1);    // P(s).V done: buffer s free again
         }
-        mbar_init(done, 1);
+        mbar_init(&done[0], 1);   // all S products complete
+        mbar_init(&done[1], 1);   // all P.V products complete
         mbar_init_fence();
     }
     if (warp == 1) {
@@ -364,7 +368,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
         if (lane == 0) {
             bool ok = true;
             int jk = 0, jv = 0;
-            uint64_t t_last = global_ns();
+            IdleWatch watch;
             while (ok && (jk < nt || jv < nt)) {
                 bool progressed = false;
                 if (jk < nt) {
@@ -391,8 +395,8 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
                     }
                 }
                 if (progressed) {
-                    t_last = global_ns();
-                } else if (aborted() || global_ns() - t_last > kWaitLimitNs) {
+                    watch.progress();
+                } else if (aborted() || watch.expired(kWaitLimitNs)) {
                     fail();
                     ok = false;
                 } else {
@@ -406,72 +410,75 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
                 if (!mbar_wait_bounded(&vfull[j % kVStages], (j / kVStages) & 1, kWaitLimitNs)) fail();
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
+        // ------------------------------------------------ S issuer
+        // S(js) as soon as K(js) has landed and the softmax has read S tile
+        // js&1 (S(js-2)): the tensor cores run up to two S tiles ahead of the
+        // softmax.  tcgen05.mma issue stalls while the pipe is full, so the
+        // P.V products have their own issuing thread (the last warp) and
+        // never wait behind an S.
         if (lane == 0) {
-            const uint32_t id_s = idesc_bf16(kQRows, kKeyTile), id_o = idesc_f16(kQRows, D);
+            const uint32_t id_s = idesc_bf16(kQRows, kKeyTile);
             const uint32_t t_qh = tmem_base + kQCol, t_ql = t_qh + uint32_t(D / 2);
             bool ok = !aborted() && mbar_wait_bounded(qfull, 0, kWaitLimitNs);
             if (!ok) fail();
             tc_fence_after();
-            // Whichever is ready: S(js) as soon as K(js) has landed and the
-            // softmax has read S buffer js&1 (S(js-2)), P(jp).V(jp) as soon as
-            // the softmax has written P(jp).  S never waits for a P.V, so the
-            // tensor cores compute the next tiles' S while the softmax works.
-            int js = 0, jp = 0;
-            uint64_t t_last = global_ns();
-            while (ok && jp < nt) {
-                bool progressed = false;
-                if (js < nt && mbar_test(&kfull[js % kKStages], (js / kKStages) & 1) &&
-                    (js < 2 || mbar_test(&sempty[js & 1], ((js >> 1) - 1) & 1))) {
-                    // S(js) = Q.K(js)^T (three hi/lo products; Q from TMEM)
-                    const int s = js & 1, ks_ = js % kKStages;
-                    tc_fence_after();
-                    const uint8_t *kst = smem + Sm::oK + ks_ * 2 * Sm::kK;
-                    const uint32_t d_s = tmem_base + kSCol + uint32_t(s * kKeyTile);
-#pragma unroll
-                    for (int ks = 0; ks < KS; ++ks) {
-                        const int bx = ks / 4, kin = ks % 4;
-                        const uint64_t kh = sw128_desc(kst + bx * kKeyTile * 128) + uint64_t(kin * 2);
-                        const uint64_t kl = sw128_desc(kst + Sm::kK + bx * kKeyTile * 128) + uint64_t(kin * 2);
-                        const uint32_t qh = t_qh + uint32_t(ks * 8), ql = t_ql + uint32_t(ks * 8);
-                        tc_mma_ts(d_s, qh, kh, id_s, ks > 0 ? 1u : 0u);
-                        tc_mma_ts(d_s, qh, kl, id_s, 1u);
-                        tc_mma_ts(d_s, ql, kh, id_s, 1u);
-                    }
-                    tc_commit(&sfull[s]);
-                    tc_commit(&kempty[ks_]);
-                    ++js;
-                    progressed = true;
-                }
-                if (jp < js && mbar_test(&pfull[jp & 1], (jp >> 1) & 1) &&
-                    mbar_test(&vfull[jp % kVStages], (jp / kVStages) & 1)) {
-                    // O += P(jp).V(jp) (P from TMEM)
-                    const int s = jp & 1, vs_ = jp % kVStages;
-                    tc_fence_after();
-                    const uint32_t d_o = tmem_base + kOCol;
-                    const uint32_t t_p = tmem_base + kPCol + uint32_t(s * (kKeyTile / 2));
-                    const uint8_t *vst = smem + Sm::oV + vs_ * Sm::kV;
-#pragma unroll
-                    for (int ks = 0; ks < PS; ++ks) {
-                        const uint64_t vd = sw128_desc(vst) + uint64_t(ks * 2);
-                        tc_mma_ts(d_o, t_p + uint32_t(ks * 8), vd, id_o, (jp > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    tc_commit(&pvdone[s]);
-                    tc_commit(&vempty[vs_]);
-                    ++jp;
-                    progressed = true;
-                }
-                if (progressed) {
-                    t_last = global_ns();
-                } else if (aborted() || global_ns() - t_last > kWaitLimitNs) {
+            for (int js = 0; ok && js < nt; ++js) {
+                const int s = js & 1, ks_ = js % kKStages;
+                if (aborted() || !mbar_wait_bounded(&kfull[ks_], (js / kKStages) & 1, kWaitLimitNs) ||
+                    (js >= 2 && !mbar_wait_bounded(&sempty[s], ((js >> 1) - 1) & 1, kWaitLimitNs))) {
                     fail();
                     ok = false;
-                } else {
-                    __nanosleep(32);   // leave the issue slots to the softmax warps
+                    break;
                 }
+                // S(js) = Q.K(js)^T (three hi/lo products; Q from TMEM; the
+                // two products with Kh are issued back to back)
+                tc_fence_after();
+                const uint8_t *kst = smem + Sm::oK + ks_ * 2 * Sm::kK;
+                const uint32_t d_s = tmem_base + kSCol + uint32_t(s * kKeyTile);
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    const int bx = ks / 4, kin = ks % 4;
+                    const uint64_t kh = sw128_desc(kst + bx * kKeyTile * 128) + uint64_t(kin * 2);
+                    const uint64_t kl = sw128_desc(kst + Sm::kK + bx * kKeyTile * 128) + uint64_t(kin * 2);
+                    const uint32_t qh = t_qh + uint32_t(ks * 8), ql = t_ql + uint32_t(ks * 8);
+                    tc_mma_ts(d_s, qh, kh, id_s, ks > 0 ? 1u : 0u);
+                    tc_mma_ts(d_s, ql, kh, id_s, 1u);
+                    tc_mma_ts(d_s, qh, kl, id_s, 1u);
+                }
+                tc_commit(&sfull[s]);
+                tc_commit(&kempty[ks_]);
             }
-            tc_commit(done);
-            if (!mbar_wait_bounded(done, 0, kWaitLimitNs)) fail();
+            tc_commit(&done[0]);
+            if (!mbar_wait_bounded(&done[0], 0, kWaitLimitNs)) fail();
+        }
+    } else if (warp == kFaPvWarp) {
+        // ------------------------------------------------ P.V issuer
+        if (lane == 0) {
+            const uint32_t id_o = idesc_f16(kQRows, D);
+            bool ok = true;
+            for (int jp = 0; ok && jp < nt; ++jp) {
+                const int s = jp & 1, vs_ = jp % kVStages;
+                if (aborted() || !mbar_wait_bounded(&pfull[s], (jp >> 1) & 1, kWaitLimitNs) ||
+                    !mbar_wait_bounded(&vfull[vs_], (jp / kVStages) & 1, kWaitLimitNs)) {
+                    fail();
+                    ok = false;
+                    break;
+                }
+                // O += P(jp).V(jp) (P from TMEM)
+                tc_fence_after();
+                const uint32_t d_o = tmem_base + kOCol;
+                const uint32_t t_p = tmem_base + kPCol + uint32_t(s * (kKeyTile / 2));
+                const uint8_t *vst = smem + Sm::oV + vs_ * Sm::kV;
+#pragma unroll
+                for (int ks = 0; ks < PS; ++ks) {
+                    const uint64_t vd = sw128_desc(vst) + uint64_t(ks * 2);
+                    tc_mma_ts(d_o, t_p + uint32_t(ks * 8), vd, id_o, (jp > 0 || ks > 0) ? 1u : 0u);
+                }
+                tc_commit(&pvdone[s]);
+                tc_commit(&vempty[vs_]);
+            }
+            tc_commit(&done[1]);
+            if (!mbar_wait_bounded(&done[1], 0, kWaitLimitNs)) fail();
         }
     } else {
         // ------------------------------------------------ softmax warps (half a query row each)

@@ -222,6 +222,24 @@ __device__ __forceinline__ void named_sync(int id, int count)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Watchdog of a polling loop: the global timer is read only while the loop
+// is idle (on its first idle pass, then every 16th), so a loop that keeps
+// making progress pays nothing for it.
+struct IdleWatch {
+    uint64_t t0 = 0;
+    uint32_t n = 0;
+    __device__ __forceinline__ void progress() { n = 0; }
+    // one idle pass; true once the loop has been idle for more than limit_ns
+    __device__ __forceinline__ bool expired(uint64_t limit_ns)
+    {
+        if (n++ == 0) {
+            t0 = global_ns();
+            return false;
+        }
+        return (n & 15) == 0 && global_ns() - t0 > limit_ns;
+    }
+};
+
 // Bounded waits give up after this long (far above any legitimate wait).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
