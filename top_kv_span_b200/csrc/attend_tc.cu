@@ -15,25 +15,26 @@
 // (fp16), from the un-rotated cache through the selection (the window is
 // never materialised in fp32).  attend_prefill_tc_kernel then runs, per
 // 128-row query block (TMEM lanes = query rows):
-//   warp 0   TMA producer: 64-key tiles of K (hi, lo) into a 4-stage ring
-//            and V^T into a 3-stage ring, each issued as soon as its stage
-//            is free (128B swizzle, no multicast)
-//   warp 1   TMEM allocation; one thread issues S(j) into one of two TMEM
-//            S tiles as soon as K(j) has landed and the tile is free
+//   warp 0   TMA producer: 128-key tiles of K (hi, lo) and V^T, each in a
+//            2-stage ring, each issued as soon as its stage is free (128B
+//            swizzle, no multicast)
+//   warp 1   TMEM allocation; one thread issues S(j) (M128 x N128 MMAs) into
+//            one of two TMEM S tiles as soon as K(j) has landed and the tile
+//            is free (its previous P.V has completed)
 //   warp 10  one thread issues O += P(j).V(j) into the TMEM O accumulator
 //            as soon as P(j) is written (a thread of its own: tcgen05.mma
 //            issue stalls while the pipe is full, and a P.V must not wait
 //            behind an S).  Both products read their A operand (the query
 //            terms, P) from TMEM, so only K and V^T come from shared memory
-//   warps 2-9 softmax: two warps per TMEM lane group, one per 32-column half
+//   warps 2-9 softmax: two warps per TMEM lane group, one per 64-column half
 //            of the S tile; first each stores its rows' query term (hi or
 //            lo) into TMEM.  A thread owns one query row's half: it reads its
-//            32 S values from TMEM, masks (causal, window end), trades its
+//            64 S values from TMEM, masks (causal, window end), trades its
 //            half-row max with the partner warp (a named barrier per pair),
 //            keeps a running reference max that moves (and rescales its half
 //            of O in TMEM) only when the row max grows by more than 2^8,
-//            stores its half of P as fp16 pairs into one of two TMEM P tiles,
-//            and finally divides its half of O by the row sum.
+//            stores its half of P as fp16 pairs over the first half of the
+//            same S tile, and finally divides its half of O by the row sum.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -54,7 +55,7 @@ constexpr int kFaSoftWarps = 8;          // two per TMEM lane group (warps 2..9)
 constexpr int kFaPvWarp = 2 + kFaSoftWarps;   // issues the P.V products
 constexpr int kFaThreads = (3 + kFaSoftWarps) * 32;
 constexpr int kQRows = 128;   // query rows per CTA (TMEM lanes)
-constexpr int kKeyTile = 64;  // keys per S tile (S columns)
+constexpr int kKeyTile = 128;  // keys per S tile (S columns, the N of its MMAs)
 constexpr float kRescaleLog2 = 8.f;
 
 struct WinMapTc {
@@ -266,8 +267,8 @@ struct FaArgs {
     int Rp, Wp;
 };
 
-constexpr int kKStages = 4;   // K tiles (hi | lo) in flight
-constexpr int kVStages = 3;   // V^T tiles in flight
+constexpr int kKStages = 2;   // K tiles (hi | lo) in flight
+constexpr int kVStages = 2;   // V^T tiles in flight
 
 // Shared-memory plan (1024-byte aligned): K stages (hi | lo) | V^T stages |
 // barriers.  The query terms and P live in TMEM.
@@ -275,16 +276,18 @@ template <int D>
 struct FaSmem {
     static constexpr int NBOX = D / 64;
     static constexpr int kK = NBOX * kKeyTile * 128;     // one of Kh / Kl
-    static constexpr int kV = D * kKeyTile * 2;          // V^T tile: D rows x 64 keys
+    static constexpr int kV = D * kKeyTile * 2;          // V^T tile: kKeyTile/64 boxes of D rows x 64 keys
     static constexpr int oK = 0, oV = kKStages * 2 * kK, oBar = oV + kVStages * kV;
     static constexpr size_t kBytes = size_t(oBar) + 32 * 8 + 1024;
 };
 
 // TMEM columns of one CTA (128 lanes = the query rows): two S tiles, the O
-// accumulator, the query terms (A operand of S: lane = row, two bf16 of the
-// head width per column) and two P tiles (A operand of P.V, two fp16 keys
-// per column).
-constexpr uint32_t kSCol = 0, kOCol = 128, kQCol = 256, kPCol = 384, kTmemCols = 512;
+// accumulator and the query terms (A operand of S: lane = row, two bf16 of
+// the head width per column).  P(j) (A operand of P.V, two fp16 keys per
+// column) overwrites the first half of its own S tile once both softmax warps
+// of the lane group have read S(j); S(j+2) goes into that tile only after
+// P(j).V(j) has completed.
+constexpr uint32_t kSCol = 0, kOCol = 2 * kKeyTile, kQCol = kOCol + 128, kTmemCols = 512;
 
 template <int D>
 __global__ void __launch_bounds__(kFaThreads, 1)
@@ -296,15 +299,14 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
     constexpr int NBOX = Sm::NBOX;
     constexpr int KS = D / 16;                 // k-steps of S over the head width
     constexpr int PS = kKeyTile / 16;          // k-steps of P.V over a key tile
-    static_assert(kOCol + D <= kQCol && kQCol + D <= kPCol && kPCol + 2 * kKeyTile / 2 <= kTmemCols,
-                  "TMEM plan");
+    static_assert(kOCol + D <= kQCol && kQCol + D <= kTmemCols, "TMEM plan");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Sm::oBar);
     uint64_t *qfull = bars, *kfull = bars + 1, *kempty = kfull + kKStages,
              *vfull = kempty + kKStages, *vempty = vfull + kVStages, *sfull = vempty + kVStages,
-             *sempty = sfull + 2, *pfull = sempty + 2, *pvdone = pfull + 2, *done = pvdone + 2;
+             *pfull = sfull + 2, *pvdone = pfull + 2, *done = pvdone + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 2);
     __shared__ int abort_flag;
 
@@ -322,9 +324,8 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sfull[s], 1);
-            mbar_init(&sempty[s], kFaSoftWarps);
-            mbar_init(&pfull[s], kFaSoftWarps);   // P buffer s written (one arrival per softmax warp)
-            mbar_init(&pvdone[s], 1);    // P(s).V done: buffer s free again
+            mbar_init(&pfull[s], kFaSoftWarps);   // P in tile s written (one arrival per softmax warp)
+            mbar_init(&pvdone[s], 1);    // P.V of tile s done: tile s free again
         }
         mbar_init(&done[0], 1);   // all S products complete
         mbar_init(&done[1], 1);   // all P.V products complete
@@ -389,7 +390,9 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
                     const int s = jv % kVStages, u = jv / kVStages;
                     if (u == 0 || mbar_test(&vempty[s], (u - 1) & 1)) {
                         mbar_arrive_expect_tx(&vfull[s], Sm::kV);
-                        tma_load_2d(smem + Sm::oV + s * Sm::kV, &vtmap, jv * kKeyTile, int(bh * D), &vfull[s]);
+                        for (int bx = 0; bx < kKeyTile / 64; ++bx)
+                            tma_load_2d(smem + Sm::oV + s * Sm::kV + bx * D * 128, &vtmap,
+                                        jv * kKeyTile + 64 * bx, int(bh * D), &vfull[s]);
                         ++jv;
                         progressed = true;
                     }
@@ -411,9 +414,8 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
         }
     } else if (warp == 1) {
         // ------------------------------------------------ S issuer
-        // S(js) as soon as K(js) has landed and the softmax has read S tile
-        // js&1 (S(js-2)): the tensor cores run up to two S tiles ahead of the
-        // softmax.  tcgen05.mma issue stalls while the pipe is full, so the
+        // S(js) as soon as K(js) has landed and S tile js&1 is free (the
+        // P(js-2).V(js-2) that read it has completed).  tcgen05.mma issue stalls while the pipe is full, so the
         // P.V products have their own issuing thread (the last warp) and
         // never wait behind an S.
         if (lane == 0) {
@@ -425,7 +427,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
             for (int js = 0; ok && js < nt; ++js) {
                 const int s = js & 1, ks_ = js % kKStages;
                 if (aborted() || !mbar_wait_bounded(&kfull[ks_], (js / kKStages) & 1, kWaitLimitNs) ||
-                    (js >= 2 && !mbar_wait_bounded(&sempty[s], ((js >> 1) - 1) & 1, kWaitLimitNs))) {
+                    (js >= 2 && !mbar_wait_bounded(&pvdone[s], ((js >> 1) - 1) & 1, kWaitLimitNs))) {
                     fail();
                     ok = false;
                     break;
@@ -467,11 +469,11 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
                 // O += P(jp).V(jp) (P from TMEM)
                 tc_fence_after();
                 const uint32_t d_o = tmem_base + kOCol;
-                const uint32_t t_p = tmem_base + kPCol + uint32_t(s * (kKeyTile / 2));
+                const uint32_t t_p = tmem_base + kSCol + uint32_t(s * kKeyTile);
                 const uint8_t *vst = smem + Sm::oV + vs_ * Sm::kV;
 #pragma unroll
                 for (int ks = 0; ks < PS; ++ks) {
-                    const uint64_t vd = sw128_desc(vst) + uint64_t(ks * 2);
+                    const uint64_t vd = sw128_desc(vst + (ks / 4) * D * 128) + uint64_t((ks % 4) * 2);
                     tc_mma_ts(d_o, t_p + uint32_t(ks * 8), vd, id_o, (jp > 0 || ks > 0) ? 1u : 0u);
                 }
                 tc_commit(&pvdone[s]);
@@ -490,7 +492,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
         __shared__ float xmax[2][4][2][32], xsum[4][2][32];
         __shared__ int xok[2][4][2];
         const int quad = warp & 3;               // TMEM lanes this warp may access
-        const int half = (warp - 2) >> 2;        // S columns [32*half, 32*half + 32)
+        const int half = (warp - 2) >> 2;        // S columns [64*half, 64*half + 64)
         const int row = quad * 32 + lane;
         const uint32_t lane_base = tmem_base + (uint32_t(quad * 32) << 16);
         const bool live = row < nrows;
@@ -538,10 +540,20 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
             float mx = -INFINITY;
             if (ok) {
                 tc_fence_after();
-                tmem_ld32(lane_base + uint32_t(s * kKeyTile + half * HC), sv);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sempty[s]);
+                {
+                    uint32_t ra[32], rb[32];
+                    const uint32_t ts = lane_base + kSCol + uint32_t(s * kKeyTile + half * HC);
+                    tmem_ld32_nowait(ts, ra);
+                    tmem_ld32_nowait(ts + 32u, rb);
+                    tmem_wait_ld();
+                    tmem_regs_after_wait(ra);
+                    tmem_regs_after_wait(rb);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        sv[i] = __uint_as_float(ra[i]);
+                        sv[32 + i] = __uint_as_float(rb[i]);
+                    }
+                }
                 // keys past this row's limit (window end, causal) are masked;
                 // halves wholly inside the limit skip the per-key test
                 const int kb = j * kKeyTile + half * HC;
@@ -561,17 +573,6 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
             pair_sync();
             if (!xok[s][quad][0] || !xok[s][quad][1]) break;   // both warps leave together
             mx = fmaxf(mx, xmax[s][quad][half ^ 1][lane]);
-            // P buffer j&1 is free once P(j-2).V(j-2) has completed
-            if (j >= 2) {
-                const bool got =
-                    !aborted() && mbar_wait_bounded(&pvdone[s], ((j - 2) >> 1) & 1, kWaitLimitNs);
-                if (!__all_sync(0xffffffffu, got)) {
-                    if (lane == 0) fail();
-                    ok = false;   // reported at the next exchange; no P or O access now
-                    continue;
-                }
-                tc_fence_after();
-            }
             const float m_new = fmaxf(m_ref, mx);
             const bool move = m_new != -INFINITY && (m_ref == -INFINITY || m_new > m_ref + kRescaleLog2);
             float fac = 1.f;
@@ -603,8 +604,11 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
                 }
             }
             // P = exp2(S - m_ref) <= 2^8 as fp16 (11-bit significand) into
-            // this row's lane of TMEM P buffer j&1: keys [32*half, 32*half+32)
-            // as 16 columns of fp16 pairs (the A operand of P.V)
+            // this row's lane of S tile j&1: keys [64*half, 64*half+64) as 32
+            // columns of fp16 pairs at columns [32*half, 32*half+32) (the A
+            // operand of P.V).  Both warps of the pair have read their S
+            // columns before the exchange above, so nothing unread is
+            // overwritten.
             const bool any_key = m_ref != -INFINITY;
             float rs = 0.f;
             float pw[HC / 2];
@@ -618,7 +622,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
                 const __half2 hv = __floats2half2_rn(p0, p1);
                 pw[e / 2] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&hv));
             }
-            tmem_st16(lane_base + kPCol + uint32_t(s * (kKeyTile / 2) + half * (HC / 2)), pw);
+            tmem_st32(lane_base + kSCol + uint32_t(s * kKeyTile + half * (HC / 2)), pw);
             l += rs;
             tc_fence_before();
             __syncwarp();
