@@ -557,16 +557,19 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
                 // keys past this row's limit (window end, causal) are masked;
                 // halves wholly inside the limit skip the per-key test
                 const int kb = j * kKeyTile + half * HC;
-                if (kb + HC - 1 <= row_lim) {
+                if (kb + HC - 1 > row_lim) {
 #pragma unroll
-                    for (int i = 0; i < HC; ++i) mx = fmaxf(mx, sv[i]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < HC; ++i) {
+                    for (int i = 0; i < HC; ++i)
                         if (kb + i > row_lim) sv[i] = -INFINITY;
-                        mx = fmaxf(mx, sv[i]);
-                    }
                 }
+                // eight independent partial maxima (short dependency chains)
+                float pm[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) pm[i] = sv[i];
+#pragma unroll
+                for (int i = 8; i < HC; ++i) pm[i & 7] = fmaxf(pm[i & 7], sv[i]);
+                mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                           fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
             }
             xmax[s][quad][half][lane] = mx;
             if (lane == 0) xok[s][quad][half] = ok ? 1 : 0;
@@ -610,7 +613,7 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
             // columns before the exchange above, so nothing unread is
             // overwritten.
             const bool any_key = m_ref != -INFINITY;
-            float rs = 0.f;
+            float rs4[4] = {0.f, 0.f, 0.f, 0.f};
             float pw[HC / 2];
 #pragma unroll
             for (int e = 0; e < HC; e += 2) {
@@ -618,10 +621,11 @@ attend_prefill_tc_kernel(const __grid_constant__ CUtensorMap khmap,
                 // yet (m_ref = -inf) has only masked keys
                 const float p0 = any_key ? ex2_approx(sv[e] - m_ref) : 0.f;
                 const float p1 = any_key ? ex2_approx(sv[e + 1] - m_ref) : 0.f;
-                rs += p0 + p1;
+                rs4[(e / 2) & 3] += p0 + p1;   // four partial sums (short chains)
                 const __half2 hv = __floats2half2_rn(p0, p1);
                 pw[e / 2] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&hv));
             }
+            const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
             tmem_st32(lane_base + kSCol + uint32_t(s * kKeyTile + half * (HC / 2)), pw);
             l += rs;
             tc_fence_before();
