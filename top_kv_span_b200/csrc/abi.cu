@@ -263,11 +263,13 @@ int reatt_step(const reatt_dims *dims, const void *q, const void *k_cache, const
     const int64_t w_known = (g.C == 1 && g.NS > 0 && !tc_attn && attn_plan(g).decode)
                                 ? decode_window_known(g)
                                 : -1;
+    bool codes = false;   // the prefill scan may leave order codes for the top-k
     cudaError_t e = launch_score_spans(g, q, k_cache, scores, ws, at(ws, p.qsum),
-                                       w_known >= 0 ? tab : nullptr, st);
+                                       w_known >= 0 ? tab : nullptr, st, true, &codes);
     if (e != cudaSuccess) return REATT_ECUDA;
     e = launch_topk(g, scores, sel, at(ws, p.topk), reinterpret_cast<uint32_t *>(at(ws, p.ticket)),
-                    int(p.ticket_bytes / sizeof(uint32_t)), w_known >= 0 ? nullptr : tab, st);
+                    int(p.ticket_bytes / sizeof(uint32_t)), w_known >= 0 ? nullptr : tab, st,
+                    codes);
     if (e != cudaSuccess) return REATT_ECUDA;
     if (tc_attn)   // many query rows: tensor-core attention
         return cuda_status(launch_attend_prefill_tc(g, q, k_cache, v_cache, k_cur, v_cur, sel, tab,

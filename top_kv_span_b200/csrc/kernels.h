@@ -42,17 +42,19 @@ int geom_of(const reatt_dims *d, Geom *g);
 // span scoring: scratch holds the fp32 summed queries when C > 1; rope_tab
 // (nullable, decode only) is filled with the step's RoPE table on the side;
 // allow_tc = false keeps C > 1 off the tensor-core scan (its tensor maps need
-// the cache's own base address)
+// the cache's own base address).  With codes_left non-null the scores may be
+// left as order codes (uint32, see order_code), which *codes_left then says;
+// otherwise they are always floats.
 size_t score_spans_ws_bytes(const Geom &geo);
 cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, float *scores,
                                void *ws, void *scratch, float2 *rope_tab, cudaStream_t st,
-                               bool allow_tc = true);
+                               bool allow_tc = true, bool *codes_left = nullptr);
 
 // prefill span scoring on tcgen05 (bf16, C > 1, S divides 32)
 bool prefill_tc_eligible(const Geom &geo);
 size_t prefill_tc_ws_bytes(const Geom &geo);
 cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, float *scores,
-                              void *ws, void *scratch, cudaStream_t st);
+                              void *ws, void *scratch, cudaStream_t st, bool *codes_left);
 
 // prefill attention on tcgen05 (bf16, more than 8 query rows per KV head)
 bool prefill_attn_tc_eligible(const Geom &geo);
@@ -64,11 +66,13 @@ cudaError_t launch_attend_prefill_tc(const Geom &geo, const void *q, const void 
 
 // top-k: scratch holds per-slice candidates when NS is large; zero_words
 // (nullable) are cleared by the first CTA (used to reset attention tickets);
-// rope_tab (nullable) is filled by spare CTAs of the same launch
+// rope_tab (nullable) is filled by spare CTAs of the same launch; with codes
+// the scores buffer holds order codes (uint32) instead of floats
 size_t topk_ws_bytes(const Geom &geo);
 int topk_selecting_ctas(const Geom &geo);   // CTAs of the first top-k launch that select
 cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void *scratch,
-                        uint32_t *zero_words, int nzero, float2 *rope_tab, cudaStream_t st);
+                        uint32_t *zero_words, int nzero, float2 *rope_tab, cudaStream_t st,
+                        bool codes = false);
 // top-k of candidate lists: per (b, h), ncand order codes and span ids (in
 // ascending id order; code 0 = empty) -> the min(k, NS) best ids, ascending
 cudaError_t launch_topk_merge(const Geom &geo, const uint32_t *codes, const int32_t *ids,

@@ -456,8 +456,9 @@ size_t score_spans_ws_bytes(const Geom &geo)
 
 cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, float *scores,
                                void *ws, void *scratch, float2 *rope_tab, cudaStream_t st,
-                               bool allow_tc)
+                               bool allow_tc, bool *codes_left)
 {
+    if (codes_left) *codes_left = false;
     if (int64_t(geo.B) * geo.Hkv * geo.NS == 0) return cudaSuccess;
     if (geo.C == 1) {
         if (geo.d == 128)
@@ -469,7 +470,7 @@ cudaError_t launch_score_spans(const Geom &geo, const void *q, const void *kc, f
     }
     if (rope_tab) return cudaErrorInvalidValue;   // only the decode scan writes the table
     if (allow_tc && prefill_tc_eligible(geo))   // tensor-core contraction (tcgen05 / TMEM)
-        return launch_prefill_tc(geo, q, kc, scores, ws, scratch, st);
+        return launch_prefill_tc(geo, q, kc, scores, ws, scratch, st, codes_left);
     float *qsum = static_cast<float *>(scratch);
     if (geo.d == 128)
         return geo_is_bf16(geo) ? launch_multi<uint16_t, 128>(geo, q, kc, scores, qsum, st)

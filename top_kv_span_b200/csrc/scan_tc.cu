@@ -270,18 +270,302 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
 }
 
+// ---------------------------------------------------------------- query-resident form
+// The same contraction with the roles of the operands swapped: two 128-query
+// tiles' terms sit in TMEM as A operands (M = 128 queries each, loaded once
+// per item) and the keys stream through a deep shared-memory ring as the B
+// operand (N = 128 tokens), so every 32 KB key tile feeds the products of
+// 256 queries: half the bytes per product that reach shared memory in the
+// key-resident form above, which the transfers from L2 bound.  An item is
+// (chunk of kQrChunk key tiles, KV head, pair of query tiles), pair fastest;
+// CTAs take items round-robin, so the query tiles of one head stream the same
+// key chunk from L2 at about the same time.  Span maxima over the item's
+// queries are folded into global order codes with atomicMax (the codes start
+// at 0, below every float's code), max over all query tiles.  Used for S = 32.
+//   warp 0  : TMA producer, one 128-token key tile per ring stage
+//   warps 1, 10: one thread each issues the products of one query slot
+//             (M128 x N128 x K16, A from TMEM) per key tile into that slot's
+//             accumulator; a barrier wait stalls the issuing thread for ~140
+//             cycles and the tensor pipe queues only an MMA or two, so each
+//             slot has its own thread: while one waits, the other's products
+//             keep the pipe busy (warp 1 also allocates TMEM)
+//   warps 2-9: warp (lane group q, slot s) stores its rows' query terms of
+//             slot s into TMEM at each item, then per key tile reduces its 32
+//             rows x 128 tokens of slot s to four span maxima (max over the
+//             tokens, then over the warp's queries) and folds them in.
+constexpr int kQrThreads = (3 + 8) * 32;   // TMA, issuer of slot 0, 8 epilogue warps, issuer of slot 1
+constexpr int kQrIssuer1 = 10;
+constexpr int kQrStages = 6;            // key tiles in flight
+constexpr int kQrChunk = 64;            // key tiles per item
+constexpr uint32_t kQrQ = 0;            // query terms of slot s at columns 128*s
+constexpr uint32_t kQrAcc = 256;        // accumulator of slot s at columns 256 + 128*s
+
+struct QrArgs {
+    int64_t items;   // nkc * BH * npair
+    int nkt;         // 128-token key tiles per head
+    int nqt;         // 128-query tiles
+    int npair;       // pairs of query tiles
+    int nterms;      // bf16 terms per query
+    int cpad;        // nqt * 128
+};
+
+template <int D>
+__global__ void __launch_bounds__(kQrThreads, 1)
+scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrArgs qa,
+                        const __nv_bfloat16 *__restrict__ terms, uint32_t *__restrict__ codes,
+                        void *ws)
+{
+    constexpr int KS = D / 16;
+    constexpr int NBOX = D / 64;
+    constexpr uint32_t kKBytes = NBOX * kBoxBytes;   // one 128-token key tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kQrStages * kKBytes);
+    uint64_t *kfull = bars, *kempty = kfull + kQrStages, *qfull = kempty + kQrStages,
+             *qempty = qfull + 2, *accfull = qempty + 2, *accempty = accfull + 2,
+             *done = accempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 2);
+    __shared__ int abort_flag;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < kQrStages; ++s) {
+            mbar_init(&kfull[s], 1);
+            mbar_init(&kempty[s], 2);     // both issuing threads commit
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&qfull[s], 4);      // slot s's query terms stored (its four warps)
+            mbar_init(&qempty[s], 1);     // the products that read slot s's terms are complete
+            mbar_init(&accfull[s], 1);
+            mbar_init(&accempty[s], 4);   // slot s's accumulator read by its four warps
+        }
+        mbar_init(&done[0], 1);
+        mbar_init(&done[1], 1);
+        mbar_init_fence();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    pdl_wait();   // the query terms and the zeroed codes come from the preceding launch
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    auto fail = [&]() {
+        report_status(ws, REATT_ETIMEOUT);
+        *(volatile int *)&abort_flag = 1;
+    };
+    auto aborted = [&]() { return *(volatile int *)&abort_flag != 0; };
+    const int BH = geo.B * geo.Hkv;
+    // item -> (key chunk, KV head, query pair) and its key tiles [k0, k1)
+    auto decode = [&](int64_t it, int64_t &bh, int &pair, int &k0, int &k1) {
+        const int64_t per_chunk = int64_t(BH) * qa.npair;
+        const int kc = int(it / per_chunk);
+        const int64_t r = it % per_chunk;
+        bh = r / qa.npair;
+        pair = int(r % qa.npair);
+        k0 = kc * kQrChunk;
+        k1 = k0 + kQrChunk < qa.nkt ? k0 + kQrChunk : qa.nkt;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t kn = 0;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; ok && it < qa.items; it += gridDim.x) {
+                int64_t bh;
+                int pair, k0, k1;
+                decode(it, bh, pair, k0, k1);
+                for (int kt = k0; kt < k1; ++kt, ++kn) {
+                    const int st = int(kn % kQrStages);
+                    const uint32_t use = kn / kQrStages;
+                    if (use > 0 && (aborted() || !mbar_wait_bounded(&kempty[st], (use - 1) & 1, kWaitLimitNs))) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    const int y = int(bh * geo.Ts + geo.G + int64_t(kt) * kTileM);
+                    mbar_arrive_expect_tx(&kfull[st], kKBytes);
+                    for (int bx = 0; bx < NBOX; ++bx)
+                        tma_load_2d(smem + st * kKBytes + bx * kBoxBytes, &kmap, 64 * bx, y, &kfull[st]);
+                }
+            }
+            for (uint32_t m = kn > kQrStages ? kn - kQrStages : 0; m < kn; ++m)
+                if (!mbar_wait_bounded(&kfull[m % kQrStages], (m / kQrStages) & 1, kWaitLimitNs)) fail();
+        }
+    } else if (warp == 1 || warp == kQrIssuer1) {
+        // ------------------------------------------------ MMA issuer of one query slot
+        if (lane == 0) {
+            const int sl = warp == 1 ? 0 : 1;
+            const uint32_t id = idesc_bf16(kTileM, kTileN);
+            const uint32_t d = tmem_base + kQrAcc + uint32_t(sl * kTileN);
+            const uint32_t tq = tmem_base + kQrQ + uint32_t(sl * 128);
+            uint32_t kn = 0, nt = 0, nq = 0;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; ok && it < qa.items; it += gridDim.x) {
+                int64_t bh;
+                int pair, k0, k1;
+                decode(it, bh, pair, k0, k1);
+                // without a second query tile, slot 1 only releases the key stages
+                const bool mine = 2 * pair + sl < qa.nqt;
+                if (mine) {
+                    if (aborted() || !mbar_wait_bounded(&qfull[sl], nq & 1, kWaitLimitNs)) {
+                        fail();
+                        break;
+                    }
+                    tc_fence_after();
+                }
+                for (int kt = k0; kt < k1; ++kt, ++kn) {
+                    const int st = int(kn % kQrStages);
+                    if (aborted() || !mbar_wait_bounded(&kfull[st], (kn / kQrStages) & 1, kWaitLimitNs) ||
+                        (mine && nt > 0 && !mbar_wait_bounded(&accempty[sl], (nt - 1) & 1, kWaitLimitNs))) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (mine) {
+                        const uint8_t *kst = smem + st * kKBytes;
+                        for (int term = 0; term < qa.nterms; ++term)
+#pragma unroll
+                            for (int ks = 0; ks < KS; ++ks) {
+                                const int bx = ks / 4, kin = ks % 4;
+                                const uint64_t kd = sw128_desc(kst + bx * kBoxBytes) + uint64_t(kin * 2);
+                                tc_mma_ts(d, tq + uint32_t(term * (D / 2) + ks * 8), kd, id,
+                                          (term | ks) != 0 ? 1u : 0u);
+                            }
+                        tc_commit(&accfull[sl]);
+                        ++nt;
+                    }
+                    tc_commit(&kempty[st]);   // this thread's products of the stage are done
+                }
+                if (!ok) break;
+                if (mine) {
+                    tc_commit(&qempty[sl]);   // the slot's terms free once this item's products are done
+                    ++nq;
+                }
+            }
+            tc_commit(&done[sl]);
+            if (!mbar_wait_bounded(&done[sl], 0, kWaitLimitNs)) fail();
+        }
+    } else {
+        // ------------------------------------------------ query terms + span maxima (256 threads)
+        const int quad = warp & 3;               // TMEM lane group: query rows [32*quad, +32)
+        const int sl = (warp - 2) >> 2;          // query slot of this warp
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = tmem_base + (uint32_t(quad * 32) << 16);
+        uint32_t nt = 0, nq = 0;
+        bool ok = true;
+        for (int64_t it = blockIdx.x; ok && it < qa.items; it += gridDim.x) {
+            int64_t bh;
+            int pair, k0, k1;
+            decode(it, bh, pair, k0, k1);
+            const int qt = 2 * pair + sl;
+            if (qt >= qa.nqt) continue;          // no second query tile in this pair
+            // this row's query terms into slot sl, once the previous item's
+            // products that read the slot are complete (rows >= C are 0)
+            if (nq > 0) {
+                const bool got = !aborted() &&
+                                 mbar_wait_bounded(&qempty[sl], (nq - 1) & 1, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) fail();
+                    break;
+                }
+                tc_fence_after();
+            }
+            for (int term = 0; term < qa.nterms; ++term) {
+                const __nv_bfloat16 *src =
+                    terms + ((bh * qa.nterms + term) * qa.cpad + int64_t(qt) * kTileN + row) * D;
+                const uint32_t tq = lane_base + kQrQ + uint32_t(sl * 128 + term * (D / 2));
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) {
+                    float w[32];
+                    const uint4 *s4 = reinterpret_cast<const uint4 *>(src + c * 64);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const uint4 v = s4[e];
+                        w[4 * e] = __uint_as_float(v.x);
+                        w[4 * e + 1] = __uint_as_float(v.y);
+                        w[4 * e + 2] = __uint_as_float(v.z);
+                        w[4 * e + 3] = __uint_as_float(v.w);
+                    }
+                    tmem_st32(tq + uint32_t(c * 32), w);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qfull[sl]);
+            ++nq;
+            const bool valid_q = qt * kTileN + row < geo.C;
+            for (int kt = k0; kt < k1; ++kt, ++nt) {
+                const bool got = !aborted() &&
+                                 mbar_wait_bounded(&accfull[sl], nt & 1, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0) fail();
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t r[4][32];
+                const uint32_t ta = lane_base + kQrAcc + uint32_t(sl * kTileN);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32_nowait(ta + uint32_t(c * 32), r[c]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_regs_after_wait(r[c]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[sl]);   // the scores are in registers
+                // four spans of 32 tokens: middle offsets t0 .. t0 + 127
+                const int64_t t0 = int64_t(kt) * kTileM;
+#pragma unroll
+                for (int sp = 0; sp < 4; ++sp) {
+                    const int64_t ts = t0 + sp * 32;
+                    float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    if (ts + 32 <= geo.M) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) pm[e & 3] = fmaxf(pm[e & 3], __uint_as_float(r[sp][e]));
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (ts + e < geo.M) pm[e & 3] = fmaxf(pm[e & 3], __uint_as_float(r[sp][e]));
+                    }
+                    float m = valid_q ? fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) : -INFINITY;
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                    if (lane == 0 && ts < geo.M && m != -INFINITY)
+                        atomicMax(&codes[bh * geo.NS + ts / 32], order_code(m));
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
 // bf16 terms of the summed group query: [BH][NT][cpad][D]; rows c >= C are 0.
 // One thread per (KV head, query, 4 consecutive dims): the group sum is formed
 // once for both terms (grid.y = KV head; 32-bit index arithmetic).
 template <int D>
 __global__ void qterms_kernel(Geom geo, const uint16_t *__restrict__ q,
-                              __nv_bfloat16 *__restrict__ out, int nterms, int cpad)
+                              __nv_bfloat16 *__restrict__ out, int nterms, int cpad,
+                              uint32_t *__restrict__ zero_codes)
 {
     constexpr int D4 = D / 4;
     const int x = blockIdx.x * blockDim.x + threadIdx.x;
+    const int bh = blockIdx.y;
+    if (zero_codes)   // span codes of the query-resident scan start below every score
+        for (int64_t s2 = x; s2 < geo.NS; s2 += int64_t(gridDim.x) * blockDim.x)
+            zero_codes[bh * geo.NS + s2] = 0u;
     if (x >= cpad * D4) return;
     const int c = x / D4, i0 = (x % D4) * 4;
-    const int bh = blockIdx.y;
     const int b = bh / geo.Hkv, h = bh % geo.Hkv;
     float v[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     if (c < geo.C) {
@@ -350,6 +634,14 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int D)
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// span scores from order codes, in place
+__global__ void decode_codes_kernel(float *__restrict__ scores, int64_t n)
+{
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += int64_t(gridDim.x) * blockDim.x)
+        scores[i] = order_decode(reinterpret_cast<const uint32_t *>(scores)[i]);
+}
+
 }  // namespace
 
 bool prefill_tc_eligible(const Geom &geo)
@@ -369,29 +661,70 @@ size_t prefill_tc_ws_bytes(const Geom &geo)
 }
 
 cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, float *scores,
-                              void *ws, void *scratch, cudaStream_t st)
+                              void *ws, void *scratch, cudaStream_t st, bool *codes_left)
 {
-    TcArgs ta;
-    ta.ntiles = int((geo.M + kTiles * kTileM - 1) / (kTiles * kTileM));
-    ta.items = int64_t(geo.B) * geo.Hkv * ta.ntiles;
-    ta.nqt = (geo.C + kTileN - 1) / kTileN;
-    ta.cpad = ta.nqt * kTileN;
-    ta.nterms = tc_terms(geo);
-    if (ta.items == 0) return cudaSuccess;
+    const int nqt = (geo.C + kTileN - 1) / kTileN;
+    const int cpad = nqt * kTileN;
+    const int nterms = tc_terms(geo);
+    const int BH = geo.B * geo.Hkv;
+    if (int64_t(BH) * geo.NS == 0) return cudaSuccess;
+    // the query-resident form serves 32-token spans (one span per 32 key columns)
+    const bool qres = geo.S == 32;
     __nv_bfloat16 *terms = static_cast<__nv_bfloat16 *>(scratch);
-    const dim3 qgrid(unsigned((ta.cpad * (geo.d / 4) + 255) / 256), unsigned(geo.B * geo.Hkv));
+    uint32_t *codes = reinterpret_cast<uint32_t *>(scores);
+    const dim3 qgrid(unsigned((cpad * (geo.d / 4) + 255) / 256), unsigned(BH));
     if (geo.d == 128)
         qterms_kernel<128><<<qgrid, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q), terms,
-                                                  ta.nterms, ta.cpad);
+                                                  nterms, cpad, qres ? codes : nullptr);
     else
         qterms_kernel<64><<<qgrid, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q), terms,
-                                                 ta.nterms, ta.cpad);
+                                                 nterms, cpad, qres ? codes : nullptr);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    CUtensorMap kmap, qmap;
-    if (!make_map(&kmap, kc, uint64_t(geo.B) * geo.Hkv * geo.Ts, geo.d) ||
-        !make_map(&qmap, terms, uint64_t(geo.B) * geo.Hkv * ta.nterms * ta.cpad, geo.d))
-        return cudaErrorInvalidValue;
+    CUtensorMap kmap;
+    if (!make_map(&kmap, kc, uint64_t(geo.B) * geo.Hkv * geo.Ts, geo.d)) return cudaErrorInvalidValue;
+    if (qres) {
+        QrArgs qa;
+        qa.nkt = int((geo.M + kTileM - 1) / kTileM);
+        qa.nqt = nqt;
+        qa.nterms = nterms;
+        qa.cpad = cpad;
+        qa.npair = (nqt + 1) / 2;
+        qa.items = int64_t((qa.nkt + kQrChunk - 1) / kQrChunk) * BH * qa.npair;
+        int grid = num_sms();
+        if (qa.items < grid) grid = int(qa.items);
+        const size_t smem = 1024 + size_t(kQrStages) * (geo.d / 64) * kBoxBytes +
+                            (2 * kQrStages + 10) * 8 + 16;
+        if (geo.d == 128) {
+            auto kern = scan_prefill_tcq_kernel<128>;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            if (e == cudaSuccess)
+                e = launch_pdl(kern, dim3(grid), dim3(kQrThreads), smem, st, kmap, geo, qa,
+                               static_cast<const __nv_bfloat16 *>(terms), codes, ws);
+        } else {
+            auto kern = scan_prefill_tcq_kernel<64>;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            if (e == cudaSuccess)
+                e = launch_pdl(kern, dim3(grid), dim3(kQrThreads), smem, st, kmap, geo, qa,
+                               static_cast<const __nv_bfloat16 *>(terms), codes, ws);
+        }
+        if (e != cudaSuccess) return e;
+        if (codes_left) {
+            *codes_left = true;   // the caller reads order codes
+        } else {
+            const int64_t n = int64_t(BH) * geo.NS;
+            decode_codes_kernel<<<unsigned((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184), 256, 0, st>>>(scores, n);
+        }
+        return cudaGetLastError();
+    }
+    TcArgs ta;
+    ta.ntiles = int((geo.M + kTiles * kTileM - 1) / (kTiles * kTileM));
+    ta.items = int64_t(BH) * ta.ntiles;
+    ta.nqt = nqt;
+    ta.cpad = cpad;
+    ta.nterms = nterms;
+    CUtensorMap qmap;
+    if (!make_map(&qmap, terms, uint64_t(BH) * ta.nterms * ta.cpad, geo.d)) return cudaErrorInvalidValue;
     int grid = num_sms();
     if (ta.items < grid) grid = int(ta.items);
     const size_t box = kBoxBytes;

@@ -58,7 +58,7 @@ __device__ void fill_rope_table(const Geom &geo, float2 *tab, int64_t chunk)
 __global__ void __launch_bounds__(kTopkThreads)
 topk_slice_kernel(Geom geo, const float *__restrict__ scores, int32_t *__restrict__ sel,
                   uint32_t *__restrict__ cand_code, int32_t *__restrict__ cand_idx, int nslices,
-                  int kkp, uint32_t *zero_words, int nzero, float2 *rope_tab)
+                  int kkp, uint32_t *zero_words, int nzero, float2 *rope_tab, int codes)
 {
     __shared__ sel::Scratch rs;
     auto bsync = [] { __syncthreads(); };
@@ -84,7 +84,8 @@ topk_slice_kernel(Geom geo, const float *__restrict__ scores, int32_t *__restric
     const int mine = n - i0 < 0 ? 0 : (n - i0 > E ? E : n - i0);
     uint32_t u[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) u[e] = e < mine ? order_code(src[i0 + e]) : 0u;
+    for (int e = 0; e < E; ++e)
+        u[e] = e < mine ? (codes ? __float_as_uint(src[i0 + e]) : order_code(src[i0 + e])) : 0u;
     const int kk = geo.k < n ? geo.k : n;
     if (nslices == 1) {
         int32_t *out = sel + bh * geo.k;
@@ -105,7 +106,7 @@ topk_slice_kernel(Geom geo, const float *__restrict__ scores, int32_t *__restric
             sel::compact_regs<kTopkThreads, E>(
                 t, u, mine, tau, take, i0, rs,
                 [&](int pos, int i) {
-                    oc[pos] = order_code(src[i]);
+                    oc[pos] = codes ? __float_as_uint(src[i]) : order_code(src[i]);
                     oi[pos] = int32_t(s_begin + i);
                 },
                 bsync);
@@ -193,7 +194,8 @@ size_t topk_ws_bytes(const Geom &geo)
 }
 
 cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void *scratch,
-                        uint32_t *zero_words, int nzero, float2 *rope_tab, cudaStream_t st)
+                        uint32_t *zero_words, int nzero, float2 *rope_tab, cudaStream_t st,
+                        bool codes)
 {
     const int BH = geo.B * geo.Hkv;
     if (geo.k == 0 && nzero == 0 && !rope_tab) return cudaSuccess;
@@ -208,7 +210,8 @@ cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void
     }
     dim3 grid(unsigned(p.nslices), unsigned(BH + tab_rows));
     cudaError_t e = launch_pdl(topk_slice_kernel, grid, dim3(kTopkThreads), 0, st, geo, scores, sel,
-                               cc, ci, p.nslices, p.kkp, zero_words, nzero, rope_tab);
+                               cc, ci, p.nslices, p.kkp, zero_words, nzero, rope_tab,
+                               codes ? 1 : 0);
     if (e != cudaSuccess) return e;
     if (p.nslices > 1 && geo.k > 0) {
         e = launch_pdl(topk_merge_kernel, dim3(BH), dim3(kTopkThreads), 0, st, geo,
