@@ -240,7 +240,37 @@ struct IdleWatch {
     }
 };
 
+// Counters in shared memory published with release and read with acquire:
+// a thread that issues tensor-core work polls one of these instead of
+// waiting on an mbarrier (an mbarrier wait stalls the issuing thread for
+// ~140 cycles even on a completed phase; this load costs a third of that).
+__device__ __forceinline__ int ld_acquire_shared(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_shared(int *p, int v)
+{
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_release_add_shared(int *p, int v)
+{
+    asm volatile("red.release.cta.shared::cta.add.s32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+
 // Bounded waits give up after this long (far above any legitimate wait).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Spin until *p >= target (acquire); false after limit_ns of waiting (the
+// global timer is read only while waiting).
+__device__ __forceinline__ bool wait_count(const int *p, int target, uint64_t limit_ns)
+{
+    if (ld_acquire_shared(p) >= target) return true;
+    IdleWatch w;
+    while (ld_acquire_shared(p) < target)
+        if (w.expired(limit_ns)) return false;
+    return true;
+}
 
 }  // namespace reatt

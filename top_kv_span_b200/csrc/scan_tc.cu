@@ -285,16 +285,23 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 //   warp 0  : TMA producer, one 128-token key tile per ring stage
 //   warps 1, 10: one thread each issues the products of one query slot
 //             (M128 x N128 x K16, A from TMEM) per key tile into that slot's
-//             accumulator; a barrier wait stalls the issuing thread for ~140
-//             cycles and the tensor pipe queues only an MMA or two, so each
-//             slot has its own thread: while one waits, the other's products
-//             keep the pipe busy (warp 1 also allocates TMEM)
+//             accumulator.  The tensor pipe queues only an MMA or two and an
+//             mbarrier wait stalls the issuing thread for ~140 cycles, so each
+//             slot has its own thread (while one waits, the other's products
+//             keep the pipe busy).  Each first reads a shared-memory counter
+//             (one acquire load): `landed` (key tiles in shared memory) or
+//             `released` (accumulator reads done); only when the count is not
+//             there yet does it wait on the matching mbarrier, which suspends
+//             the thread instead of spinning.  Warp 1 also allocates TMEM.
+//   warp 11 : waits on each key stage's TMA barrier in order and publishes
+//             the landed count
 //   warps 2-9: warp (lane group q, slot s) stores its rows' query terms of
 //             slot s into TMEM at each item, then per key tile reduces its 32
 //             rows x 128 tokens of slot s to four span maxima (max over the
 //             tokens, then over the warp's queries) and folds them in.
-constexpr int kQrThreads = (3 + 8) * 32;   // TMA, issuer of slot 0, 8 epilogue warps, issuer of slot 1
+constexpr int kQrThreads = (4 + 8) * 32;   // TMA, issuer 0, 8 epilogue warps, issuer 1, watcher
 constexpr int kQrIssuer1 = 10;
+constexpr int kQrWatcher = 11;
 constexpr int kQrStages = 6;            // key tiles in flight
 constexpr int kQrChunk = 64;            // key tiles per item
 constexpr uint32_t kQrQ = 0;            // query terms of slot s at columns 128*s
@@ -327,10 +334,13 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
              *done = accempty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 2);
     __shared__ int abort_flag;
+    __shared__ int landed, released[2];   // key tiles landed; accumulator reads done (per slot)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         abort_flag = 0;
+        landed = 0;
+        released[0] = released[1] = 0;
         for (int s = 0; s < kQrStages; ++s) {
             mbar_init(&kfull[s], 1);
             mbar_init(&kempty[s], 2);     // both issuing threads commit
@@ -422,8 +432,12 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
                 }
                 for (int kt = k0; kt < k1; ++kt, ++kn) {
                     const int st = int(kn % kQrStages);
-                    if (aborted() || !mbar_wait_bounded(&kfull[st], (kn / kQrStages) & 1, kWaitLimitNs) ||
-                        (mine && nt > 0 && !mbar_wait_bounded(&accempty[sl], (nt - 1) & 1, kWaitLimitNs))) {
+                    // key tile kn landed; slot's previous accumulator read by its four warps
+                    if (aborted() ||
+                        (ld_acquire_shared(&landed) < int(kn) + 1 &&
+                         !mbar_wait_bounded(&kfull[st], (kn / kQrStages) & 1, kWaitLimitNs)) ||
+                        (mine && nt > 0 && ld_acquire_shared(&released[sl]) < 4 * int(nt) &&
+                         !mbar_wait_bounded(&accempty[sl], (nt - 1) & 1, kWaitLimitNs))) {
                         fail();
                         ok = false;
                         break;
@@ -452,6 +466,26 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
             }
             tc_commit(&done[sl]);
             if (!mbar_wait_bounded(&done[sl], 0, kWaitLimitNs)) fail();
+        }
+    } else if (warp == kQrWatcher) {
+        // ------------------------------------------------ landed count of the key ring
+        if (lane == 0) {
+            uint32_t kn = 0;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; ok && it < qa.items; it += gridDim.x) {
+                int64_t bh;
+                int pair, k0, k1;
+                decode(it, bh, pair, k0, k1);
+                for (int kt = k0; kt < k1; ++kt, ++kn) {
+                    if (aborted() ||
+                        !mbar_wait_bounded(&kfull[kn % kQrStages], (kn / kQrStages) & 1, kWaitLimitNs)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    st_release_shared(&landed, int(kn) + 1);
+                }
+            }
         }
     } else {
         // ------------------------------------------------ query terms + span maxima (256 threads)
@@ -520,7 +554,10 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
                 for (int c = 0; c < 4; ++c) tmem_regs_after_wait(r[c]);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&accempty[sl]);   // the scores are in registers
+                if (lane == 0) {   // the scores are in registers
+                    red_release_add_shared(&released[sl], 1);
+                    mbar_arrive(&accempty[sl]);
+                }
                 // four spans of 32 tokens: middle offsets t0 .. t0 + 127
                 const int64_t t0 = int64_t(kt) * kTileM;
 #pragma unroll
