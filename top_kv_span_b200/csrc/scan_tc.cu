@@ -558,8 +558,10 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
                     red_release_add_shared(&released[sl], 1);
                     mbar_arrive(&accempty[sl]);
                 }
-                // four spans of 32 tokens: middle offsets t0 .. t0 + 127
+                // four spans of 32 tokens: middle offsets t0 .. t0 + 127; this
+                // row's max over each span's tokens
                 const int64_t t0 = int64_t(kt) * kTileM;
+                float m[4];
 #pragma unroll
                 for (int sp = 0; sp < 4; ++sp) {
                     const int64_t ts = t0 + sp * 32;
@@ -572,11 +574,23 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
                         for (int e = 0; e < 32; ++e)
                             if (ts + e < geo.M) pm[e & 3] = fmaxf(pm[e & 3], __uint_as_float(r[sp][e]));
                     }
-                    float m = valid_q ? fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) : -INFINITY;
-#pragma unroll
-                    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                    if (lane == 0 && ts < geo.M && m != -INFINITY)
-                        atomicMax(&codes[bh * geo.NS + ts / 32], order_code(m));
+                    m[sp] = valid_q ? fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) : -INFINITY;
+                }
+                // max over the warp's 32 rows for all four spans at once: two
+                // halving exchanges leave each lane one span (2*bit4 + bit3 of
+                // its lane id), three more finish the max over all rows
+                const bool u16 = (lane & 16) != 0, u8 = (lane & 8) != 0;
+                float a0 = u16 ? m[2] : m[0], a1 = u16 ? m[3] : m[1];
+                a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, u16 ? m[0] : m[2], 16));
+                a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, u16 ? m[1] : m[3], 16));
+                float mx = fmaxf(u8 ? a1 : a0, __shfl_xor_sync(0xffffffffu, u8 ? a0 : a1, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                if ((lane & 7) == 0) {
+                    const int64_t ts = t0 + (2 * int(u16) + int(u8)) * 32;
+                    if (ts < geo.M && mx != -INFINITY)
+                        atomicMax(&codes[bh * geo.NS + ts / 32], order_code(mx));
                 }
             }
         }
