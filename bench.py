@@ -45,7 +45,7 @@ METRIC = "ReAttention step latency (µs) and KV-scan GB/s vs HBM peak at 128K–
 PROFILE_SUMMARY = {
     "llama3_8b_128k": os.path.join(ROOT, "profiles", "scan_decode_llama3_8b_128k.md"),
     "llama3_8b_prefill_256k": os.path.join(ROOT, "profiles",
-                                           "scan_prefill_tc_llama3_8b_prefill_64k.md"),
+                                           "scan_prefill_tcq_llama3_8b_prefill_64k.md"),
     "qwen2_1p5b_4m": os.path.join(ROOT, "profiles", "scan_decode_qwen2_1p5b_4m.md"),
 }
 # key of the traffic line in a summary (a smaller capture scaled to the workload)
@@ -202,7 +202,8 @@ def roofline(w, scan_b, scan_ms):
         return {"bound": "tensor", "achieved": round(achieved, 1), "peak": tflops,
                 "peak_kind": kind + " (bf16 burst)", "unit": "TFLOP/s",
                 "frac": round(achieved / tflops, 4), "traffic": traffic,
-                "kernel": "scan_prefill_tc_kernel", "flops_per_launch": scan_flops(w),
+                "kernel": "scan_prefill_tcq_kernel" if w.S == 32 else "scan_prefill_tc_kernel",
+                "flops_per_launch": scan_flops(w),
                 "note": "issued MMA work is 2x (bf16 hi + lo query terms)"}
     achieved = scan_b / (scan_ms * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "peak_kind": kind,
