@@ -67,6 +67,18 @@ CASES = {
                                              L=64, S=8, k=30, n_needles=0, seed=25),
     "prefill_bf16_s64_fallback": LLAMA.replace(name="s64", Hq=4, Hkv=1, C=9, T=3000, G=8, L=64,
                                                S=64, k=5, n_needles=0, seed=26),
+    # query-resident tensor-core scan (S = 32): d = 64; one raw query head per KV
+    # head (one term); two raw heads and an odd number of query tiles (an item
+    # with one query slot); several key chunks per head with a 3-token last key
+    # tile and a 3-token last span
+    "prefill_bf16_d64_s32_c200": LLAMA.replace(name="c200", Hq=8, Hkv=2, d=64, C=200, T=7000,
+                                               G=8, L=100, S=32, k=12, n_needles=2, seed=31),
+    "prefill_bf16_g1_s32_c260": LLAMA.replace(name="c260", Hq=2, Hkv=2, C=260, T=6003, G=8,
+                                              L=64, S=32, k=10, n_needles=2, seed=32),
+    "prefill_bf16_g2_s32_c300": LLAMA.replace(name="c300s32", Hq=4, Hkv=2, C=300, T=5000, G=8,
+                                              L=100, S=32, k=12, n_needles=1, seed=34),
+    "prefill_bf16_chunks_c130": LLAMA.replace(name="c130k", Hq=8, Hkv=2, C=130, T=20003, G=32,
+                                              L=256, S=32, k=16, n_needles=3, seed=33),
     "two_level_topk": LLAMA.replace(name="big_ns", Hq=2, Hkv=1, d=64, T=200000, G=32, L=256,
                                     S=8, k=100, n_needles=4, seed=21),
     "batch3_large_s": TINY.replace(name="b3", B=3, Hq=2, Hkv=1, T=5000, G=2, L=40, S=100, k=3,
