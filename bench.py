@@ -47,9 +47,12 @@ PROFILE_SUMMARY = {
     "llama3_8b_prefill_256k": os.path.join(ROOT, "profiles",
                                            "scan_prefill_tcq_llama3_8b_prefill_64k.md"),
     "qwen2_1p5b_4m": os.path.join(ROOT, "profiles", "scan_decode_qwen2_1p5b_4m.md"),
+    "llama3_8b_1m_x4": os.path.join(ROOT, "profiles", "scan_decode_llama3_8b_1m.md"),
+    "tiny_f32_4k": os.path.join(ROOT, "profiles", "scan_decode_tiny_f32_4k.md"),
 }
 # key of the traffic line in a summary (a smaller capture scaled to the workload)
-PROFILE_KEY = {"llama3_8b_prefill_256k": "traffic_bytes_per_launch_256k:"}
+PROFILE_KEY = {"llama3_8b_prefill_256k": "traffic_bytes_per_launch_256k:",
+               "llama3_8b_1m_x4": "traffic_bytes_per_launch_1m_x4:"}
 
 
 def step_bytes(w):

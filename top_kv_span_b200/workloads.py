@@ -87,6 +87,11 @@ WORKLOADS = {
         S=32, k=64, dtype="bf16", rope_base=5e5, seed=1005, n_needles=0, dist="channel",
         description="the 2048-query prefill chunk over a 64K cache: K+V 268 MB (more than "
                     "L2), the size full profiler captures of the prefill kernels run on"),
+    "llama3_8b_1m": Workload(
+        "llama3_8b_1m", B=1, Hq=32, Hkv=8, d=128, C=1, T=1048576, G=32, L=4096, S=32, k=64,
+        dtype="bf16", rope_base=5e5, seed=1006, n_needles=8, dist="channel",
+        description="one sequence of the 1M x 4 decode (K+V 4.3 GB): the size profiler "
+                    "captures of its scan run on"),
     "qwen2_1p5b_4m": Workload(
         "qwen2_1p5b_4m", B=1, Hq=12, Hkv=2, d=128, C=1, T=4194304, G=32, L=4096, S=32, k=64,
         dtype="bf16", rope_base=1e6, seed=1004, n_needles=5, dist="channel",
