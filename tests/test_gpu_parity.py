@@ -169,7 +169,7 @@ def test_topk_sizes_and_value_spreads(R, dist):
     counts, k around and above the span count, and several heads at once."""
     rng = np.random.default_rng(["normal", "ties", "narrow", "equal", "wide"].index(dist) + 40)
     for NS, k in [(1, 1), (7, 3), (7, 9), (100, 64), (3967, 64), (4096, 64), (4097, 64),
-                  (5000, 1), (9000, 200), (20000, 64), (2048, 2048)]:
+                  (5000, 1), (8192, 64), (8193, 64), (9000, 200), (20000, 64), (2048, 2048)]:
         w = LLAMA.replace(B=2, Hq=4, Hkv=2, d=64, T=32 + 4096 + 32 * NS, G=32, L=4096, S=32, k=k)
         d = R.dims_of(w)
         assert R.reatt_num_spans(d) == NS

@@ -13,10 +13,13 @@
 // generic select of 4 passes of 8 bits read from memory.  A stable block
 // compaction in index order then writes the chosen ids, which are therefore
 // already ascending -- no sort is needed.
-// NS <= kSlice: one CTA per head.  Larger NS: slice CTAs (kSlice scores each)
-// emit their own top-k candidates in index order, and one merge CTA per head
-// runs the same select on the candidates.  The global top-k under the total
-// order (score desc, id asc) is always inside the union of the slices' top-k.
+// NS <= 4096: one CTA per head, 8 codes per thread; NS <= 8192: one CTA per
+// head, 16 codes per thread (no second launch).  Larger NS: slice CTAs (4096
+// scores each, 8 codes per thread: faster than 8192-score slices and a
+// smaller merge) emit their own top-k candidates in index order, and one
+// merge CTA per head runs the same select on the candidates.  The global
+// top-k under the total order (score desc, id asc) is always inside the union
+// of the slices' top-k.
 #include "common.cuh"
 #include "kernels.h"
 #include "select.cuh"
@@ -29,8 +32,9 @@ namespace {
 #define REATT_TOPK_THREADS 512
 #endif
 constexpr int kTopkThreads = REATT_TOPK_THREADS;
-constexpr int kSlice = 4096;
-constexpr int kMaxE = 16;   // codes per thread of the register path
+constexpr int kSlice = 4096;        // 8 codes per thread: small heads and every slice
+constexpr int kSliceWide = 8192;    // 16 codes per thread: the largest head one CTA takes
+constexpr int kMaxE = 16;           // codes per thread of the register path
 
 // cos/sin table of the window positions: tab[p*(d/2) + i] = (cos, sin) of
 // p * base^(-2i/d), for p < Wmax.  Filled by spare CTAs of the top-k launch,
@@ -55,6 +59,7 @@ __device__ void fill_rope_table(const Geom &geo, float2 *tab, int64_t chunk)
     }
 }
 
+template <int E>
 __global__ void __launch_bounds__(kTopkThreads)
 topk_slice_kernel(Geom geo, const float *__restrict__ scores, int32_t *__restrict__ sel,
                   uint32_t *__restrict__ cand_code, int32_t *__restrict__ cand_idx, int nslices,
@@ -75,11 +80,11 @@ topk_slice_kernel(Geom geo, const float *__restrict__ scores, int32_t *__restric
     if (zero_words && slice == 0 && bh == 0)
         for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero_words[i] = 0u;
 
-    const int64_t s_begin = int64_t(slice) * kSlice;
-    int n = int(geo.NS - s_begin < kSlice ? geo.NS - s_begin : kSlice);
+    constexpr int kS = E * kTopkThreads;   // scores of one slice
+    const int64_t s_begin = int64_t(slice) * kS;
+    int n = int(geo.NS - s_begin < kS ? geo.NS - s_begin : kS);
     if (n < 0) n = 0;
     const float *src = scores + bh * geo.NS + s_begin;
-    constexpr int E = kSlice / kTopkThreads;
     const int i0 = int(threadIdx.x) * E;
     const int mine = n - i0 < 0 ? 0 : (n - i0 > E ? E : n - i0);
     uint32_t u[E];
@@ -161,11 +166,13 @@ topk_merge_kernel(Geom geo, const uint32_t *__restrict__ cand_code,
 
 struct TopkPlan {
     int nslices, kkp;
+    bool wide;   // one CTA with 16 codes per thread (4096 < NS <= 8192)
 };
 TopkPlan topk_plan(const Geom &geo)
 {
     TopkPlan p;
-    p.nslices = geo.NS <= kSlice ? 1 : int((geo.NS + kSlice - 1) / kSlice);
+    p.wide = geo.NS > kSlice && geo.NS <= kSliceWide;
+    p.nslices = geo.NS <= kSliceWide ? 1 : int((geo.NS + kSlice - 1) / kSlice);
     p.kkp = geo.k < kSlice ? geo.k : kSlice;
     return p;
 }
@@ -209,9 +216,13 @@ cudaError_t launch_topk(const Geom &geo, const float *scores, int32_t *sel, void
         tab_rows = (chunks + p.nslices - 1) / p.nslices;
     }
     dim3 grid(unsigned(p.nslices), unsigned(BH + tab_rows));
-    cudaError_t e = launch_pdl(topk_slice_kernel, grid, dim3(kTopkThreads), 0, st, geo, scores, sel,
-                               cc, ci, p.nslices, p.kkp, zero_words, nzero, rope_tab,
-                               codes ? 1 : 0);
+    cudaError_t e =
+        p.wide ? launch_pdl(topk_slice_kernel<kSliceWide / kTopkThreads>, grid, dim3(kTopkThreads),
+                            0, st, geo, scores, sel, cc, ci, p.nslices, p.kkp, zero_words, nzero,
+                            rope_tab, codes ? 1 : 0)
+               : launch_pdl(topk_slice_kernel<kSlice / kTopkThreads>, grid, dim3(kTopkThreads), 0,
+                            st, geo, scores, sel, cc, ci, p.nslices, p.kkp, zero_words, nzero,
+                            rope_tab, codes ? 1 : 0);
     if (e != cudaSuccess) return e;
     if (p.nslices > 1 && geo.k > 0) {
         e = launch_pdl(topk_merge_kernel, dim3(BH), dim3(kTopkThreads), 0, st, geo,
