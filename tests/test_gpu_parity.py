@@ -79,6 +79,8 @@ CASES = {
                                               L=100, S=32, k=12, n_needles=1, seed=34),
     "prefill_bf16_chunks_c130": LLAMA.replace(name="c130k", Hq=8, Hkv=2, C=130, T=20003, G=32,
                                               L=256, S=32, k=16, n_needles=3, seed=33),
+    "prefill_bf16_b2_c150": LLAMA.replace(name="b2c150", B=2, Hq=4, Hkv=2, C=150, T=4000, G=8,
+                                          L=100, S=32, k=8, n_needles=2, seed=35),
     "two_level_topk": LLAMA.replace(name="big_ns", Hq=2, Hkv=1, d=64, T=200000, G=32, L=256,
                                     S=8, k=100, n_needles=4, seed=21),
     "batch3_large_s": TINY.replace(name="b3", B=3, Hq=2, Hkv=1, T=5000, G=2, L=40, S=100, k=3,
