@@ -277,11 +277,13 @@ scan_prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 // operand (N = 128 tokens), so every 32 KB key tile feeds the products of
 // 256 queries: half the bytes per product that reach shared memory in the
 // key-resident form above, which the transfers from L2 bound.  An item is
-// (chunk of kQrChunk key tiles, KV head, pair of query tiles), pair fastest;
+// (chunk of key tiles, KV head, pair of query tiles), pair fastest;
 // CTAs take items round-robin, so the query tiles of one head stream the same
 // key chunk from L2 at about the same time.  Span maxima over the item's
 // queries are folded into global order codes with atomicMax (the codes start
 // at 0, below every float's code), max over all query tiles.  Used for S = 32.
+// The chunk is sized for about six items per CTA (32 to 128 key tiles): larger
+// items reload the query terms less often, smaller ones balance the last wave.
 //   warp 0  : TMA producer, one 128-token key tile per ring stage
 //   warps 1, 10: one thread each issues the products of one query slot
 //             (M128 x N128 x K16, A from TMEM) per key tile into that slot's
@@ -303,12 +305,13 @@ constexpr int kQrThreads = (4 + 8) * 32;   // TMA, issuer 0, 8 epilogue warps, i
 constexpr int kQrIssuer1 = 10;
 constexpr int kQrWatcher = 11;
 constexpr int kQrStages = 6;            // key tiles in flight
-constexpr int kQrChunk = 64;            // key tiles per item
+constexpr int kQrChunkMin = 32, kQrChunkMax = 128;   // key tiles per item
 constexpr uint32_t kQrQ = 0;            // query terms of slot s at columns 128*s
 constexpr uint32_t kQrAcc = 256;        // accumulator of slot s at columns 256 + 128*s
 
 struct QrArgs {
     int64_t items;   // nkc * BH * npair
+    int chunk;       // key tiles per item
     int nkt;         // 128-token key tiles per head
     int nqt;         // 128-query tiles
     int npair;       // pairs of query tiles
@@ -378,8 +381,8 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
         const int64_t r = it % per_chunk;
         bh = r / qa.npair;
         pair = int(r % qa.npair);
-        k0 = kc * kQrChunk;
-        k1 = k0 + kQrChunk < qa.nkt ? k0 + kQrChunk : qa.nkt;
+        k0 = kc * qa.chunk;
+        k1 = k0 + qa.chunk < qa.nkt ? k0 + qa.chunk : qa.nkt;
     };
 
     if (warp == 0) {
@@ -741,8 +744,13 @@ cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, fl
         qa.nterms = nterms;
         qa.cpad = cpad;
         qa.npair = (nqt + 1) / 2;
-        qa.items = int64_t((qa.nkt + kQrChunk - 1) / kQrChunk) * BH * qa.npair;
         int grid = num_sms();
+        {
+            const int64_t per_tile = int64_t(BH) * qa.npair;   // items per key chunk
+            int64_t c = int64_t(qa.nkt) * per_tile / (int64_t(grid) * 6);
+            qa.chunk = int(c < kQrChunkMin ? kQrChunkMin : (c > kQrChunkMax ? kQrChunkMax : c));
+            qa.items = int64_t((qa.nkt + qa.chunk - 1) / qa.chunk) * per_tile;
+        }
         if (qa.items < grid) grid = int(qa.items);
         const size_t smem = 1024 + size_t(kQrStages) * (geo.d / 64) * kBoxBytes +
                             (2 * kQrStages + 10) * 8 + 16;
