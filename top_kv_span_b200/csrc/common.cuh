@@ -262,15 +262,4 @@ __device__ __forceinline__ void red_release_add_shared(int *p, int v)
 // Bounded waits give up after this long (far above any legitimate wait).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Spin until *p >= target (acquire); false after limit_ns of waiting (the
-// global timer is read only while waiting).
-__device__ __forceinline__ bool wait_count(const int *p, int target, uint64_t limit_ns)
-{
-    if (ld_acquire_shared(p) >= target) return true;
-    IdleWatch w;
-    while (ld_acquire_shared(p) < target)
-        if (w.expired(limit_ns)) return false;
-    return true;
-}
-
 }  // namespace reatt

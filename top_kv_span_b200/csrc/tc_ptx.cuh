@@ -220,24 +220,6 @@ constexpr uint32_t idesc_f16(int M, int N)
 // Instruction descriptor as idesc_bf16 with A read MN-major (transposed).
 constexpr uint32_t idesc_bf16_amn(int M, int N) { return idesc_bf16(M, N) | (1u << 15); }
 
-// Per-thread 16-byte asynchronous copy global -> shared (L2 only), and the
-// mbarrier arrival that fires once all of this thread's earlier copies have
-// landed (counted against the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async16(void *dst, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all()
-{
-    asm volatile("cp.async.wait_all;" ::: "memory");
-}
-
 // Generic-proxy shared-memory writes made visible to the async proxy (the
 // tensor core reads operands through it).
 __device__ __forceinline__ void fence_proxy_async_smem()
