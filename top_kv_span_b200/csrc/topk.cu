@@ -29,7 +29,7 @@ namespace reatt {
 namespace {
 
 #ifndef REATT_TOPK_THREADS
-#define REATT_TOPK_THREADS 512
+#define REATT_TOPK_THREADS 1024
 #endif
 constexpr int kTopkThreads = REATT_TOPK_THREADS;
 constexpr int kSlice = 4096;        // 8 codes per thread: small heads and every slice
