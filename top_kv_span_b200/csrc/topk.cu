@@ -13,10 +13,10 @@
 // generic select of 4 passes of 8 bits read from memory.  A stable block
 // compaction in index order then writes the chosen ids, which are therefore
 // already ascending -- no sort is needed.
-// NS <= 4096: one CTA per head, 8 codes per thread; NS <= 8192: one CTA per
-// head, 16 codes per thread (no second launch).  Larger NS: slice CTAs (4096
-// scores each, 8 codes per thread: faster than 8192-score slices and a
-// smaller merge) emit their own top-k candidates in index order, and one
+// CTAs of 1024 threads.  NS <= 4096: one CTA per head, 4 codes per thread;
+// NS <= 8192: one CTA per head, 8 codes per thread (no second launch).
+// Larger NS: slice CTAs (4096 scores each, 4 codes per thread: faster than
+// 8192-score slices and a smaller merge) emit their own top-k candidates in index order, and one
 // merge CTA per head runs the same select on the candidates.  The global
 // top-k under the total order (score desc, id asc) is always inside the union
 // of the slices' top-k.
@@ -32,9 +32,9 @@ namespace {
 #define REATT_TOPK_THREADS 1024
 #endif
 constexpr int kTopkThreads = REATT_TOPK_THREADS;
-constexpr int kSlice = 4096;        // 8 codes per thread: small heads and every slice
-constexpr int kSliceWide = 8192;    // 16 codes per thread: the largest head one CTA takes
-constexpr int kMaxE = 16;           // codes per thread of the register path
+constexpr int kSlice = 4096;        // 4 codes per thread: small heads and every slice
+constexpr int kSliceWide = 8192;    // 8 codes per thread: the largest head one CTA takes
+constexpr int kMaxE = 16;           // codes per thread of the merge's register path
 
 // cos/sin table of the window positions: tab[p*(d/2) + i] = (cos, sin) of
 // p * base^(-2i/d), for p < Wmax.  Filled by spare CTAs of the top-k launch,
@@ -166,7 +166,7 @@ topk_merge_kernel(Geom geo, const uint32_t *__restrict__ cand_code,
 
 struct TopkPlan {
     int nslices, kkp;
-    bool wide;   // one CTA with 16 codes per thread (4096 < NS <= 8192)
+    bool wide;   // one CTA with 8 codes per thread (4096 < NS <= 8192)
 };
 TopkPlan topk_plan(const Geom &geo)
 {
