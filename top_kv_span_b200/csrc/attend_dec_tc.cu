@@ -14,9 +14,12 @@
 //   warp 0      TMA: the tile's K and V rows in boxes of 32 or 8 rows x 64
 //               columns, 128B-swizzled, each inside one run of the window (the
 //               global part, a chosen span, the local part, the current tokens)
-//               and one 32-row quarter of the tile, which has its own barrier;
-//               lane q issues quarter q, so the four quarters' loads go out
-//               together; V lands directly in the MN-major operand layout
+//               and one 32-row quarter of the tile; lane q issues quarter q, so
+//               the four quarters' loads go out together.  K quarters have a
+//               barrier each, V one per stage; a tile's K goes out when its
+//               raw stage is free and its V when its V stage is free, so the
+//               chosen rows' keys load as soon as the selection is in.  V lands
+//               directly in the MN-major operand layout
 //   warp 1      TMEM allocation; one thread issues S(j) and then P(j-1).V(j-1)
 //   warps 2-9   rotate the raw keys of each quarter as it lands (RoPE with
 //               the step's cos/sin table) and split them into the hi/lo
@@ -115,9 +118,11 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
     uint64_t *rawempty = bars + 2, *vempty = bars + 4, *kopfull = bars + 6,
              *kopempty = bars + 7, *sfull = bars + 8, *sempty = bars + 10, *pfull = bars + 12,
              *pvdone = bars + 13, *done = bars + 14, *qready = bars + 15;
-    // loads of stage s, rows [32q, 32q + 32): tq[4s + q]
+    // K rows [32q, 32q + 32) of stage s: tq[4s + q]
     uint64_t *tq = bars + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 24);
+    // V rows of stage s: tv[s]
+    uint64_t *tv = bars + 26;
     __shared__ float red[2][kDtSoftWarps][RP], lred[kDtSoftWarps][RP];
     __shared__ float f_m[RP], f_l[RP];
     __shared__ __align__(16) float s_acc[RP * D];
@@ -141,6 +146,7 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
         mbar_init(done, 1);
         mbar_init(qready, kDtSoftWarps);
         for (int q = 0; q < 8; ++q) mbar_init(&tq[q], 1);
+        for (int q = 0; q < 2; ++q) mbar_init(&tv[q], 1);
         mbar_init_fence();
     }
     if (warp == 1) {
@@ -234,94 +240,133 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
             prefetch_tensormap(&maps.kq);
             prefetch_tensormap(&maps.vq);
         }
-        bool ok = true;
-        for (int j = 0; j < nt; ++j) {
+        // Lane q (< 4) issues the boxes of quarter q (rows [32q, 32q + 32)) of
+        // tile j: its K rows (want_v false) or its V rows, each box inside one
+        // run of the window.  V gets 8 more rows past an odd number of 8-row
+        // groups so P.V runs whole 16-key steps.
+        auto issue_quarter = [&](int j, int q, bool want_v) {
             const int s = j & 1;
-            if (j == nE) {
-                __syncwarp();
-                pdl_wait();   // the global and chosen rows need the selection
-                if (sel_cached)
-                    for (int x = lane; x < jn; x += 32) sel_s[x] = sel_bh[j0 + x];
-                __syncwarp();
-            }
-            if (j >= 2) {
-                const uint32_t par = uint32_t((j >> 1) - 1) & 1u;
-                ok = ok && !aborted() && mbar_wait_bounded(&rawempty[s], par, kWaitLimitNs) &&
-                     mbar_wait_bounded(&vempty[s], par, kWaitLimitNs);
-            }
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) fail();
-                break;
-            }
-            if (lane < 4) {
-                // lane q issues quarter q (rows [32q, 32q + 32) of the tile):
-                // its expected bytes, then its boxes
-                const int q = lane;
-                int p0, n;
-                tile_at(j, p0, n);
-                const int ng = (n + 7) / 8;
-                {
-                    int rows = 8 * ng - kDtQuarter * q;
-                    rows = rows < 0 ? 0 : (rows > kDtQuarter ? kDtQuarter : rows);
-                    uint32_t bytes = uint32_t(rows) * 512u;
-                    if ((ng & 1) && (8 * ng) / kDtQuarter == q) bytes += 8u * 256u;
-                    if (bytes)
-                        mbar_arrive_expect_tx(&tq[4 * s + q], bytes);
-                    else
-                        mbar_arrive(&tq[4 * s + q]);
+            int p0, n;
+            tile_at(j, p0, n);
+            uint8_t *dst = smem + (want_v ? Sm::oV : Sm::oRaw) + s * kDtTile;
+            uint64_t *bar = want_v ? &tv[s] : &tq[4 * s + q];
+            const int r_end = kDtQuarter * q + kDtQuarter < n ? kDtQuarter * q + kDtQuarter : n;
+            for (int r = kDtQuarter * q; r < r_end;) {
+                const int p = p0 + r;
+                int run_end;
+                bool cur = false;
+                int64_t y;
+                if (p < g_end) {
+                    run_end = g_end;
+                    y = bh * geo.Ts + p;
+                } else if (p - g_end < nsel) {
+                    const int qq = p - g_end, jj = qq / geo.S, off = qq - jj * geo.S;
+                    int sp = sel_cached ? sel_s[jj - j0] : sel_bh[jj];
+                    sp = sp < 0 ? 0 : (sp >= int(geo.NS) ? int(geo.NS) - 1 : sp);
+                    run_end = g_end + (jj + 1) * geo.S;
+                    y = bh * geo.Ts + geo.G + int64_t(sp) * geo.S + off;
+                } else if (p - g_end - nsel < nloc) {
+                    run_end = g_end + nsel + nloc;
+                    y = bh * geo.Ts + m.loc_begin + (p - g_end - nsel);
+                } else {
+                    run_end = int(W);
+                    cur = true;
+                    y = bh * geo.C + (p - g_end - nsel - nloc);
                 }
-                uint8_t *kst = smem + Sm::oRaw + s * kDtTile, *vst = smem + Sm::oV + s * kDtTile;
-                const int r_end = kDtQuarter * q + kDtQuarter < n ? kDtQuarter * q + kDtQuarter : n;
-                uint64_t *bar = &tq[4 * s + q];
-                for (int r = kDtQuarter * q; r < r_end;) {
-                    const int p = p0 + r;
-                    int run_end;
-                    bool cur = false;
-                    int64_t y;
-                    if (p < g_end) {
-                        run_end = g_end;
-                        y = bh * geo.Ts + p;
-                    } else if (p - g_end < nsel) {
-                        const int qq = p - g_end, jj = qq / geo.S, off = qq - jj * geo.S;
-                        int sp = sel_cached ? sel_s[jj - j0] : sel_bh[jj];
-                        sp = sp < 0 ? 0 : (sp >= int(geo.NS) ? int(geo.NS) - 1 : sp);
-                        run_end = g_end + (jj + 1) * geo.S;
-                        y = bh * geo.Ts + geo.G + int64_t(sp) * geo.S + off;
-                    } else if (p - g_end - nsel < nloc) {
-                        run_end = g_end + nsel + nloc;
-                        y = bh * geo.Ts + m.loc_begin + (p - g_end - nsel);
-                    } else {
-                        run_end = int(W);
-                        cur = true;
-                        y = bh * geo.C + (p - g_end - nsel - nloc);
+                int len = (run_end < p0 + r_end ? run_end : p0 + r_end) - p;
+                while (len > 0) {
+                    const int hs = (!cur && len >= 32 && (r & 31) == 0) ? 0 : 1;
+                    const CUtensorMap *mp = want_v ? (cur ? &maps.vq : &maps.v[hs])
+                                                   : (cur ? &maps.kq : &maps.k[hs]);
+                    tma_load_2d(dst + r * 128, mp, 0, int(y), bar);
+                    tma_load_2d(dst + kDtHalf + r * 128, mp, 64, int(y), bar);
+                    r += dt_box_rows(hs);
+                    if (want_v && r >= n && (r & 8)) {
+                        tma_load_2d(dst + r * 128, mp, 0, int(y), bar);
+                        tma_load_2d(dst + kDtHalf + r * 128, mp, 64, int(y), bar);
                     }
-                    int len = (run_end < p0 + r_end ? run_end : p0 + r_end) - p;
-                    while (len > 0) {
-                        const int hs = (!cur && len >= 32 && (r & 31) == 0) ? 0 : 1;
-                        const CUtensorMap *km = cur ? &maps.kq : &maps.k[hs];
-                        const CUtensorMap *vm = cur ? &maps.vq : &maps.v[hs];
-                        tma_load_2d(kst + r * 128, km, 0, int(y), bar);
-                        tma_load_2d(kst + kDtHalf + r * 128, km, 64, int(y), bar);
-                        tma_load_2d(vst + r * 128, vm, 0, int(y), bar);
-                        tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), bar);
-                        r += dt_box_rows(hs);
-                        if (r >= n && (r & 8)) {
-                            tma_load_2d(vst + r * 128, vm, 0, int(y), bar);
-                            tma_load_2d(vst + kDtHalf + r * 128, vm, 64, int(y), bar);
-                        }
-                        y += dt_box_rows(hs);
-                        len -= dt_box_rows(hs);
-                    }
+                    y += dt_box_rows(hs);
+                    len -= dt_box_rows(hs);
                 }
             }
-            __syncwarp();
+        };
+        // K of tile jk once its raw stage is free (tile jk - 2 converted) and,
+        // from tile nE on, the selection is in; V of tile jv (jv < jk) once
+        // its V stage is free (P.V of tile jv - 2 done).  Neither waits for
+        // the other, so the chosen rows' keys load as soon as the selection
+        // lands, not after the second-last tile's P.V.
+        bool ok = true, sel_in = nE >= nt;
+        int jk = 0, jv = 0;
+        IdleWatch watch;
+        while (jv < nt) {
+            bool progressed = false;
+            if (jv < jk) {
+                bool ready = jv < 2 || mbar_test(&vempty[jv & 1], uint32_t((jv >> 1) - 1) & 1u);
+                ready = __shfl_sync(0xffffffffu, ready, 0);
+                if (ready) {
+                    int p0, n;
+                    tile_at(jv, p0, n);
+                    const int ng = (n + 7) / 8;
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(&tv[jv & 1], uint32_t(8 * (ng + (ng & 1))) * 256u);
+                    __syncwarp();
+                    if (lane < 4) issue_quarter(jv, lane, true);
+                    __syncwarp();
+                    ++jv;
+                    progressed = true;
+                }
+            }
+            if (jk < nt) {
+                bool ready = true;
+                if (jk == nE && !sel_in) {   // the global and chosen rows need the selection
+                    __syncwarp();
+                    pdl_wait();
+                    sel_in = true;
+                    if (sel_cached)
+                        for (int x = lane; x < jn; x += 32) sel_s[x] = sel_bh[j0 + x];
+                    __syncwarp();
+                }
+                if (jk >= 2)
+                    ready = mbar_test(&rawempty[jk & 1], uint32_t((jk >> 1) - 1) & 1u);
+                ready = __shfl_sync(0xffffffffu, ready, 0);
+                if (ready) {
+                    if (lane < 4) {
+                        int p0, n;
+                        tile_at(jk, p0, n);
+                        const int ng = (n + 7) / 8;
+                        int rows = 8 * ng - kDtQuarter * lane;
+                        rows = rows < 0 ? 0 : (rows > kDtQuarter ? kDtQuarter : rows);
+                        uint64_t *bar = &tq[4 * (jk & 1) + lane];
+                        if (rows)
+                            mbar_arrive_expect_tx(bar, uint32_t(rows) * 256u);
+                        else
+                            mbar_arrive(bar);
+                        issue_quarter(jk, lane, false);
+                    }
+                    __syncwarp();
+                    ++jk;
+                    progressed = true;
+                }
+            }
+            if (progressed) {
+                watch.progress();
+            } else {
+                if (__any_sync(0xffffffffu, aborted() || watch.expired(kWaitLimitNs))) {
+                    ok = false;
+                    break;
+                }
+                __nanosleep(32);
+            }
         }
+        if (!ok && lane == 0) fail();
         // drain: the last loads of each stage have landed
-        for (int j = nt - 2 < 0 ? 0 : nt - 2; ok && j < nt; ++j)
+        for (int j = nt - 2 < 0 ? 0 : nt - 2; ok && j < nt; ++j) {
+            const uint32_t par = uint32_t(j >> 1) & 1u;
+            bool got = mbar_wait_bounded(&tv[j & 1], par, kWaitLimitNs);
             for (int q = 0; q < 4; ++q)
-                if (!mbar_wait_bounded(&tq[4 * (j & 1) + q], uint32_t(j >> 1) & 1u, kWaitLimitNs) &&
-                    lane == 0)
-                    fail();
+                got = mbar_wait_bounded(&tq[4 * (j & 1) + q], par, kWaitLimitNs) && got;
+            if (!got && lane == 0) fail();
+        }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -361,10 +406,7 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
                     progressed = true;
                 }
                 if (jp < js && mbar_test(pfull, uint32_t(jp) & 1u) &&
-                    mbar_test(&tq[4 * (jp & 1)], uint32_t(jp >> 1) & 1u) &&
-                    mbar_test(&tq[4 * (jp & 1) + 1], uint32_t(jp >> 1) & 1u) &&
-                    mbar_test(&tq[4 * (jp & 1) + 2], uint32_t(jp >> 1) & 1u) &&
-                    mbar_test(&tq[4 * (jp & 1) + 3], uint32_t(jp >> 1) & 1u)) {
+                    mbar_test(&tv[jp & 1], uint32_t(jp >> 1) & 1u)) {
                     const int s = jp & 1;
                     int p0, n;
                     tile_at(jp, p0, n);
