@@ -439,7 +439,8 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
         // ------------------------------------------------ RoPE + hi/lo split of K
         // All converter warps take each 32-row quarter as soon as it lands:
         // thread = (key kq of the quarter, pair chunk c); the key's cos/sin
-        // come from the step's table, loaded one quarter ahead.
+        // come from the step's table for a tile's first quarter (loaded one
+        // quarter ahead) and by rotation for the others.
         const int ct = tid - kDtConvBase * 32;
         const int c = ct & 7;                    // pairs 8c..8c+7 (dims and dims + 64)
         const int kq = ct >> 3;                  // 0..31
@@ -463,6 +464,24 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
 #pragma unroll
         for (int e = 0; e < 8; ++e) nx[e] = make_float2(1.f, 0.f);
         if (nt > 0) anchors(0, nx);
+        // (cos, sin) of 32 positions at this thread's frequencies: the key of
+        // quarter q + 1 sits 32 positions after that of quarter q, so its
+        // angles are the previous ones rotated by these (angle addition in
+        // fp32, three steps at most) and the table is read once per tile.
+        // Row 32 of the table exists whenever a tile has more than 32 rows.
+        float2 r32[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r32[e] = make_float2(1.f, 0.f);
+        if (geo.Wmax > kDtQuarter) {
+            const float4 *tr =
+                reinterpret_cast<const float4 *>(a.tab + int64_t(kDtQuarter) * (D / 2) + 8 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 t = __ldcg(tr + e);
+                r32[2 * e] = make_float2(t.x, t.y);
+                r32[2 * e + 1] = make_float2(t.z, t.w);
+            }
+        }
         bool ok = true;
         uint8_t *kh = smem + Sm::oKh, *kl = smem + Sm::oKl;
         for (int j = 0; j < nt && ok; ++j) {
@@ -475,7 +494,16 @@ attend_decode_tc_kernel(const __grid_constant__ DtMaps maps, Geom geo, AttnArgs 
 #pragma unroll
                 for (int e = 0; e < 8; ++e) cs[e] = nx[e];
                 const int job = 4 * j + qd;
-                if (job + 1 < 4 * nt) anchors(job + 1, nx);
+                if (job + 1 < 4 * nt) {
+                    if (qd < 3) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            nx[e] = make_float2(fmaf(cs[e].x, r32[e].x, -cs[e].y * r32[e].y),
+                                                fmaf(cs[e].y, r32[e].x, cs[e].x * r32[e].y));
+                    } else {
+                        anchors(job + 1, nx);
+                    }
+                }
                 ok = ok && !aborted() &&
                      mbar_wait_bounded(&tq[4 * s + qd], uint32_t(j >> 1) & 1u, kWaitLimitNs) &&
                      (qd > 0 || j == 0 || mbar_wait_bounded(kopempty, uint32_t(j - 1) & 1u, kWaitLimitNs));
