@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "select.cuh"
 #include "tc_ptx.cuh"
 
 namespace reatt {
@@ -306,6 +307,7 @@ constexpr int kQrIssuer1 = 10;
 constexpr int kQrWatcher = 11;
 constexpr int kQrStages = 6;            // key tiles in flight
 constexpr int kQrChunkMin = 32, kQrChunkMax = 128;   // key tiles per item
+constexpr int kQrFilterChunk = 8;                     // listed key tiles per item (exact pass)
 constexpr uint32_t kQrQ = 0;            // query terms of slot s at columns 128*s
 constexpr uint32_t kQrAcc = 256;        // accumulator of slot s at columns 256 + 128*s
 
@@ -315,8 +317,13 @@ struct QrArgs {
     int nkt;         // 128-token key tiles per head
     int nqt;         // 128-query tiles
     int npair;       // pairs of query tiles
-    int nterms;      // bf16 terms per query
+    int nterms;      // bf16 terms per query used by the products
+    int tstride;     // terms per query in the terms buffer (>= nterms)
     int cpad;        // nqt * 128
+    // Optional tile list: key tile kt of head bh is tile tiles[bh*nkt + kt],
+    // for kt < ntile[bh] only (null: kt itself, for every kt < nkt).
+    const int32_t *tiles;
+    const int32_t *ntile;
 };
 
 template <int D>
@@ -382,7 +389,12 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
         bh = r / qa.npair;
         pair = int(r % qa.npair);
         k0 = kc * qa.chunk;
-        k1 = k0 + qa.chunk < qa.nkt ? k0 + qa.chunk : qa.nkt;
+        const int kend = qa.ntile ? __ldg(qa.ntile + bh) : qa.nkt;
+        k1 = k0 + qa.chunk < kend ? k0 + qa.chunk : kend;
+    };
+    // key tile kt of head bh
+    auto tile_of = [&](int64_t bh, int kt) {
+        return qa.tiles ? __ldg(qa.tiles + bh * qa.nkt + kt) : kt;
     };
 
     if (warp == 0) {
@@ -394,7 +406,7 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
                 int64_t bh;
                 int pair, k0, k1;
                 decode(it, bh, pair, k0, k1);
-                for (int kt = k0; kt < k1; ++kt, ++kn) {
+                for (int kt = k0; kt < k1; ++kt, ++kn) {   // (an empty item issues nothing)
                     const int st = int(kn % kQrStages);
                     const uint32_t use = kn / kQrStages;
                     if (use > 0 && (aborted() || !mbar_wait_bounded(&kempty[st], (use - 1) & 1, kWaitLimitNs))) {
@@ -402,7 +414,7 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
                         ok = false;
                         break;
                     }
-                    const int y = int(bh * geo.Ts + geo.G + int64_t(kt) * kTileM);
+                    const int y = int(bh * geo.Ts + geo.G + int64_t(tile_of(bh, kt)) * kTileM);
                     mbar_arrive_expect_tx(&kfull[st], kKBytes);
                     for (int bx = 0; bx < NBOX; ++bx)
                         tma_load_2d(smem + st * kKBytes + bx * kBoxBytes, &kmap, 64 * bx, y, &kfull[st]);
@@ -424,6 +436,7 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
                 int64_t bh;
                 int pair, k0, k1;
                 decode(it, bh, pair, k0, k1);
+                if (k0 >= k1) continue;   // empty item (tile list): skipped by every role
                 // without a second query tile, slot 1 only releases the key stages
                 const bool mine = 2 * pair + sl < qa.nqt;
                 if (mine) {
@@ -502,6 +515,7 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
             int64_t bh;
             int pair, k0, k1;
             decode(it, bh, pair, k0, k1);
+            if (k0 >= k1) continue;              // empty item (tile list)
             const int qt = 2 * pair + sl;
             if (qt >= qa.nqt) continue;          // no second query tile in this pair
             // this row's query terms into slot sl, once the previous item's
@@ -517,7 +531,7 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
             }
             for (int term = 0; term < qa.nterms; ++term) {
                 const __nv_bfloat16 *src =
-                    terms + ((bh * qa.nterms + term) * qa.cpad + int64_t(qt) * kTileN + row) * D;
+                    terms + ((bh * qa.tstride + term) * qa.cpad + int64_t(qt) * kTileN + row) * D;
                 const uint32_t tq = lane_base + kQrQ + uint32_t(sl * 128 + term * (D / 2));
 #pragma unroll
                 for (int c = 0; c < D / 64; ++c) {
@@ -563,7 +577,7 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
                 }
                 // four spans of 32 tokens: middle offsets t0 .. t0 + 127; this
                 // row's max over each span's tokens
-                const int64_t t0 = int64_t(kt) * kTileM;
+                const int64_t t0 = int64_t(tile_of(bh, kt)) * kTileM;
                 float m[4];
 #pragma unroll
                 for (int sp = 0; sp < 4; ++sp) {
@@ -610,7 +624,7 @@ scan_prefill_tcq_kernel(const __grid_constant__ CUtensorMap kmap, Geom geo, QrAr
 template <int D>
 __global__ void qterms_kernel(Geom geo, const uint16_t *__restrict__ q,
                               __nv_bfloat16 *__restrict__ out, int nterms, int cpad,
-                              uint32_t *__restrict__ zero_codes)
+                              uint32_t *__restrict__ zero_codes, uint32_t *__restrict__ qnorm)
 {
     constexpr int D4 = D / 4;
     const int x = blockIdx.x * blockDim.x + threadIdx.x;
@@ -650,6 +664,7 @@ __global__ void qterms_kernel(Geom geo, const uint16_t *__restrict__ q,
             }
         }
     }
+    float ss[2] = {0.f, 0.f};   // squares of the stored hi and lo terms
     for (int term = 0; term < nterms; ++term) {
         __nv_bfloat162 lo2 = __floats2bfloat162_rn(v[term][0], v[term][1]);
         __nv_bfloat162 hi2 = __floats2bfloat162_rn(v[term][2], v[term][3]);
@@ -657,7 +672,158 @@ __global__ void qterms_kernel(Geom geo, const uint16_t *__restrict__ q,
         w.x = *reinterpret_cast<const uint32_t *>(&lo2);
         w.y = *reinterpret_cast<const uint32_t *>(&hi2);
         *reinterpret_cast<uint2 *>(out + ((int64_t(bh) * nterms + term) * cpad + c) * D + i0) = w;
+        const float e0 = bf16lo(w.x), e1 = bf16hi(w.x), e2 = bf16lo(w.y), e3 = bf16hi(w.y);
+        ss[term & 1] += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
     }
+    if (qnorm) {   // max over the chunk's queries of ||q_hi|| and ||q_lo|| (D4 lanes per query)
+        __shared__ float wmax[2][32];
+#pragma unroll
+        for (int o = D4 / 2; o >= 1; o >>= 1) {
+            ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], o);
+            ss[1] += __shfl_xor_sync(0xffffffffu, ss[1], o);
+        }
+        float n0 = sqrtf(ss[0]), n1 = sqrtf(ss[1]);
+#pragma unroll
+        for (int o = D4; o < 32; o <<= 1) {   // the warp's other queries
+            n0 = fmaxf(n0, __shfl_xor_sync(0xffffffffu, n0, o));
+            n1 = fmaxf(n1, __shfl_xor_sync(0xffffffffu, n1, o));
+        }
+        const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+        if ((threadIdx.x & 31) == 0) {
+            wmax[0][warp] = n0;
+            wmax[1][warp] = n1;
+        }
+        __syncthreads();   // whole blocks reach here (cpad * D4 is a multiple of 256)
+        if (threadIdx.x == 0) {   // non-negative floats order like their bit patterns
+            for (int w2 = 1; w2 < nw; ++w2) {
+                n0 = fmaxf(n0, wmax[0][w2]);
+                n1 = fmaxf(n1, wmax[1][w2]);
+            }
+            atomicMax(qnorm + 2 * bh, __float_as_uint(n0));
+            atomicMax(qnorm + 2 * bh + 1, __float_as_uint(n1));
+        }
+    }
+}
+
+// ---------------------------------------------------------------- two-pass filter
+// The fused step needs only the selection, so with hi/lo query terms the
+// scan runs twice: once with the hi terms alone over every key tile, and
+// once with hi + lo over the key tiles that hold a span the first pass
+// cannot rule out.  For a query c and key t the two passes' products differ
+// by q_lo[c].k_t plus the rounding of two fp32 accumulations, so a span's
+// exact maximum lies within E_sp = (max_c ||q_lo[c]|| + a 2^-14 max_c
+// ||q_hi[c]|| rounding allowance) * max_{t in sp} ||k_t|| of its hi-only
+// maximum.  A span whose upper bound stays below the k-th largest lower
+// bound cannot be among the k largest exact maxima (each of the k spans with
+// the largest lower bounds has an exact maximum at least that large), so
+// only the other spans' tiles are scanned again, with the same products as
+// the one-pass scan.
+
+// kn[bh][sp] = max over the span's tokens of ||k_t||_2 (fp32); block 0 also
+// clears the per-head query norms that qterms_kernel raises.  One warp per
+// span of 32 tokens, each load a contiguous 512 (D = 128) or 256 bytes.
+template <int D>
+__global__ void __launch_bounds__(256)
+span_knorm_kernel(Geom geo, const uint16_t *__restrict__ kc, float *__restrict__ kn,
+                  uint32_t *__restrict__ qnorm)
+{
+    constexpr int CPT = D * 2 / 16;   // 16-byte chunks per token
+    constexpr int TPL = 32 / CPT;     // tokens per warp load
+    const int lane = threadIdx.x & 31;
+    const int64_t BH = int64_t(geo.B) * geo.Hkv;
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < 2 * BH; i += blockDim.x) qnorm[i] = 0u;
+    const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (wid >= BH * geo.NS) return;   // whole warps
+    const int64_t bh = wid / geo.NS, sp = wid % geo.NS;
+    const int64_t t0 = sp * 32;       // middle offset of the span's first token
+    const uint4 *src = reinterpret_cast<const uint4 *>(kc + (bh * geo.Ts + geo.G + t0) * D);
+    float mx = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < CPT; ++j) {
+        const int tok = j * TPL + lane / CPT;
+        float ss = 0.f;
+        if (t0 + tok < geo.M) {
+            const uint4 w = __ldg(src + j * 32 + lane);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float a0 = bf16lo(ws[e]), a1 = bf16hi(ws[e]);
+                ss = fmaf(a0, a0, fmaf(a1, a1, ss));
+            }
+        }
+#pragma unroll
+        for (int o = CPT / 2; o >= 1; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        mx = fmaxf(mx, ss);
+    }
+#pragma unroll
+    for (int o = 16; o >= CPT; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) kn[bh * geo.NS + sp] = sqrtf(mx);
+}
+
+constexpr int kCandThreads = 1024;
+constexpr int kCandE = 8;             // spans per thread: NS <= 8192, key tiles <= 2048
+
+// One CTA per (b, KV head): from the hi-only span codes, the span key norms
+// and the query norms, the list of key tiles (ascending) that hold a span
+// whose upper bound reaches the k-th largest lower bound; every span code is
+// then reset to 0 for the exact pass.
+__global__ void __launch_bounds__(kCandThreads)
+prefill_candidates_kernel(Geom geo, uint32_t *__restrict__ codes, const float *__restrict__ kn,
+                          const uint32_t *__restrict__ qnorm, int32_t *__restrict__ tiles,
+                          int32_t *__restrict__ ntile, int nkt)
+{
+    __shared__ sel::Scratch rs;
+    __shared__ uint32_t tmask[kCandThreads * kCandE / 4 / 32];
+    auto bsync = [] { __syncthreads(); };
+    const int t = threadIdx.x;
+    const int64_t bh = blockIdx.x;
+    const int NS = int(geo.NS);
+    for (int i = t; i < kCandThreads * kCandE / 4 / 32; i += kCandThreads) tmask[i] = 0u;
+    const float qh = __uint_as_float(qnorm[2 * bh]), ql = __uint_as_float(qnorm[2 * bh + 1]);
+    // bound per unit key norm; the 2^-10 factors cover the norms' own fp32 rounding
+    const float unit = (ql * 1.0009765625f + qh * 6.103515625e-05f) * 1.0009765625f;
+    const int i0 = t * kCandE;
+    const int mine = NS - i0 < 0 ? 0 : (NS - i0 > kCandE ? kCandE : NS - i0);
+    uint32_t *hc = codes + bh * NS;
+    uint32_t lbc[kCandE];
+    float ub[kCandE];
+#pragma unroll
+    for (int e = 0; e < kCandE; ++e) {
+        lbc[e] = 0u;
+        ub[e] = -INFINITY;
+        if (e < mine) {
+            const uint32_t c = hc[i0 + e];
+            const float ap = c ? order_decode(c) : -INFINITY;
+            const float E = __fmul_ru(unit, kn[bh * NS + i0 + e]);
+            lbc[e] = order_code(__fsub_rd(ap, E));
+            ub[e] = __fadd_ru(ap, E);
+        }
+    }
+    __syncthreads();   // the tile mask is clear
+    uint32_t tau, take;
+    const uint32_t kk = uint32_t(geo.k < NS ? geo.k : NS);
+    sel::select_regs<kCandThreads, kCandE>(t, lbc, mine, kk, rs, tau, take, bsync);
+    const float tauf = order_decode(tau);
+#pragma unroll
+    for (int e = 0; e < kCandE; ++e)
+        if (e < mine && ub[e] >= tauf) {
+            const int tl = (i0 + e) >> 2;   // 4 spans of 32 tokens per 128-token tile
+            atomicOr(&tmask[tl >> 5], 1u << (tl & 31));
+        }
+#pragma unroll
+    for (int e = 0; e < kCandE; ++e)
+        if (e < mine) hc[i0 + e] = 0u;
+    __syncthreads();
+    const int ta = 2 * t, tb = 2 * t + 1;
+    const int ma = ta < nkt && ((tmask[ta >> 5] >> (ta & 31)) & 1u);
+    const int mb = tb < nkt && ((tmask[tb >> 5] >> (tb & 31)) & 1u);
+    int total;
+    const int pos = sel::exclusive_sum<kCandThreads>(t, ma + mb, rs, &total, bsync);
+    int32_t *tl = tiles + bh * nkt;
+    if (ma) tl[pos] = ta;
+    if (mb) tl[pos + ma] = tb;
+    if (t == 0) ntile[bh] = total;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
@@ -707,11 +873,49 @@ bool prefill_tc_eligible(const Geom &geo)
 
 static int tc_terms(const Geom &geo) { return geo.g <= 2 ? geo.g : 2; }
 
+static size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// The two-pass filter serves the fused step's query-resident scan with hi/lo
+// query terms when one CTA can rank a head's spans.
+static bool filter_eligible(const Geom &geo)
+{
+    return geo.S == 32 && geo.g > 2 && tc_terms(geo) == 2 && geo.NS <= kCandThreads * kCandE &&
+           geo.k > 0 && geo.k < geo.NS;
+}
+
+static size_t terms_bytes(const Geom &geo)
+{
+    const int cpad = (geo.C + kTileN - 1) / kTileN * kTileN;
+    return size_t(geo.B) * geo.Hkv * tc_terms(geo) * cpad * geo.d * sizeof(__nv_bfloat16);
+}
+
+// Filter workspace after the terms: span key norms [BH][NS], query norms
+// [BH][2], key tile lists [BH][nkt], list lengths [BH].
+struct FilterWs {
+    float *kn;
+    uint32_t *qnorm;
+    int32_t *tiles, *ntile;
+};
+static size_t filter_ws(const Geom &geo, void *scratch, FilterWs *f)
+{
+    const size_t BH = size_t(geo.B) * geo.Hkv;
+    const size_t nkt = size_t((geo.M + kTileM - 1) / kTileM);
+    size_t off = up256(terms_bytes(geo));
+    uint8_t *base = static_cast<uint8_t *>(scratch);
+    if (f) f->kn = reinterpret_cast<float *>(base + off);
+    off = up256(off + BH * geo.NS * sizeof(float));
+    if (f) f->qnorm = reinterpret_cast<uint32_t *>(base + off);
+    off = up256(off + 2 * BH * sizeof(uint32_t));
+    if (f) f->tiles = reinterpret_cast<int32_t *>(base + off);
+    off = up256(off + BH * nkt * sizeof(int32_t));
+    if (f) f->ntile = reinterpret_cast<int32_t *>(base + off);
+    return off + BH * sizeof(int32_t);
+}
+
 size_t prefill_tc_ws_bytes(const Geom &geo)
 {
     if (!prefill_tc_eligible(geo)) return 0;
-    const int cpad = (geo.C + kTileN - 1) / kTileN * kTileN;
-    return size_t(geo.B) * geo.Hkv * tc_terms(geo) * cpad * geo.d * sizeof(__nv_bfloat16);
+    return filter_eligible(geo) ? filter_ws(geo, nullptr, nullptr) : terms_bytes(geo);
 }
 
 cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, float *scores,
@@ -726,13 +930,29 @@ cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, fl
     const bool qres = geo.S == 32;
     __nv_bfloat16 *terms = static_cast<__nv_bfloat16 *>(scratch);
     uint32_t *codes = reinterpret_cast<uint32_t *>(scores);
+    // the fused step (which reads only the selection) takes the two-pass filter
+    const bool two = qres && codes_left && filter_eligible(geo);
+    FilterWs fw{};
+    if (two) {
+        filter_ws(geo, scratch, &fw);
+        const int64_t threads = int64_t(BH) * geo.NS * 32;
+        const unsigned blocks = unsigned((threads + 255) / 256);
+        if (geo.d == 128)
+            span_knorm_kernel<128><<<blocks, 256, 0, st>>>(geo, static_cast<const uint16_t *>(kc),
+                                                           fw.kn, fw.qnorm);
+        else
+            span_knorm_kernel<64><<<blocks, 256, 0, st>>>(geo, static_cast<const uint16_t *>(kc),
+                                                          fw.kn, fw.qnorm);
+    }
     const dim3 qgrid(unsigned((cpad * (geo.d / 4) + 255) / 256), unsigned(BH));
     if (geo.d == 128)
         qterms_kernel<128><<<qgrid, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q), terms,
-                                                  nterms, cpad, qres ? codes : nullptr);
+                                                  nterms, cpad, qres ? codes : nullptr,
+                                                  two ? fw.qnorm : nullptr);
     else
         qterms_kernel<64><<<qgrid, 256, 0, st>>>(geo, static_cast<const uint16_t *>(q), terms,
-                                                 nterms, cpad, qres ? codes : nullptr);
+                                                 nterms, cpad, qres ? codes : nullptr,
+                                                 two ? fw.qnorm : nullptr);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     CUtensorMap kmap;
@@ -741,33 +961,56 @@ cudaError_t launch_prefill_tc(const Geom &geo, const void *q, const void *kc, fl
         QrArgs qa;
         qa.nkt = int((geo.M + kTileM - 1) / kTileM);
         qa.nqt = nqt;
-        qa.nterms = nterms;
+        qa.nterms = two ? 1 : nterms;   // the filter's first pass: hi terms only
+        qa.tstride = nterms;
         qa.cpad = cpad;
         qa.npair = (nqt + 1) / 2;
-        int grid = num_sms();
+        qa.tiles = nullptr;
+        qa.ntile = nullptr;
+        const int64_t per_tile = int64_t(BH) * qa.npair;   // items per key chunk
         {
-            const int64_t per_tile = int64_t(BH) * qa.npair;   // items per key chunk
-            int64_t c = int64_t(qa.nkt) * per_tile / (int64_t(grid) * 6);
+            int64_t c = int64_t(qa.nkt) * per_tile / (int64_t(num_sms()) * 6);
             qa.chunk = int(c < kQrChunkMin ? kQrChunkMin : (c > kQrChunkMax ? kQrChunkMax : c));
             qa.items = int64_t((qa.nkt + qa.chunk - 1) / qa.chunk) * per_tile;
         }
-        if (qa.items < grid) grid = int(qa.items);
         const size_t smem = 1024 + size_t(kQrStages) * (geo.d / 64) * kBoxBytes +
                             (2 * kQrStages + 10) * 8 + 16;
-        if (geo.d == 128) {
-            auto kern = scan_prefill_tcq_kernel<128>;
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-            if (e == cudaSuccess)
-                e = launch_pdl(kern, dim3(grid), dim3(kQrThreads), smem, st, kmap, geo, qa,
-                               static_cast<const __nv_bfloat16 *>(terms), codes, ws);
-        } else {
-            auto kern = scan_prefill_tcq_kernel<64>;
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-            if (e == cudaSuccess)
-                e = launch_pdl(kern, dim3(grid), dim3(kQrThreads), smem, st, kmap, geo, qa,
-                               static_cast<const __nv_bfloat16 *>(terms), codes, ws);
-        }
+        auto run = [&](const QrArgs &a) {
+            int grid = num_sms();
+            if (a.items < grid) grid = int(a.items);
+            cudaError_t r;
+            if (geo.d == 128) {
+                auto kern = scan_prefill_tcq_kernel<128>;
+                r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+                if (r == cudaSuccess)
+                    r = launch_pdl(kern, dim3(grid), dim3(kQrThreads), smem, st, kmap, geo, a,
+                                   static_cast<const __nv_bfloat16 *>(terms), codes, ws);
+            } else {
+                auto kern = scan_prefill_tcq_kernel<64>;
+                r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+                if (r == cudaSuccess)
+                    r = launch_pdl(kern, dim3(grid), dim3(kQrThreads), smem, st, kmap, geo, a,
+                                   static_cast<const __nv_bfloat16 *>(terms), codes, ws);
+            }
+            return r;
+        };
+        e = run(qa);
         if (e != cudaSuccess) return e;
+        if (two) {
+            // candidate key tiles, then the exact products over them only
+            prefill_candidates_kernel<<<unsigned(BH), kCandThreads, 0, st>>>(
+                geo, codes, fw.kn, fw.qnorm, fw.tiles, fw.ntile, qa.nkt);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            QrArgs q2 = qa;
+            q2.nterms = nterms;
+            q2.tiles = fw.tiles;
+            q2.ntile = fw.ntile;
+            q2.chunk = kQrFilterChunk;
+            q2.items = int64_t((qa.nkt + q2.chunk - 1) / q2.chunk) * per_tile;
+            e = run(q2);
+            if (e != cudaSuccess) return e;
+        }
         if (codes_left) {
             *codes_left = true;   // the caller reads order codes
         } else {

@@ -1,5 +1,5 @@
 // Block-wide k-th-largest selection on order codes, shared by the top-k
-// kernels and the decode scan (which selects inside its own CTAs).
+// kernels and the prefill scan's candidate filter.
 //
 // Every helper runs on NT participating threads with thread index t in
 // [0, NT) and a barrier functor `sync` that synchronises exactly those
