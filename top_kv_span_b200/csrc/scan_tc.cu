@@ -307,7 +307,7 @@ constexpr int kQrIssuer1 = 10;
 constexpr int kQrWatcher = 11;
 constexpr int kQrStages = 6;            // key tiles in flight
 constexpr int kQrChunkMin = 32, kQrChunkMax = 128;   // key tiles per item
-constexpr int kQrFilterChunk = 8;                     // listed key tiles per item (exact pass)
+constexpr int kQrFilterChunk = 16;                    // listed key tiles per item (exact pass)
 constexpr uint32_t kQrQ = 0;            // query terms of slot s at columns 128*s
 constexpr uint32_t kQrAcc = 256;        // accumulator of slot s at columns 256 + 128*s
 
