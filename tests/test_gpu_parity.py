@@ -81,12 +81,14 @@ CASES = {
                                               L=256, S=32, k=16, n_needles=3, seed=33),
     "prefill_bf16_b2_c150": LLAMA.replace(name="b2c150", B=2, Hq=4, Hkv=2, C=150, T=4000, G=8,
                                           L=100, S=32, k=8, n_needles=2, seed=35),
-    # GQA 4 with hi/lo query terms: the step's two-pass span filter, with two
-    # sequences, and with k a large share of the spans (many candidates)
-    "prefill_bf16_b2_g4_c150": LLAMA.replace(name="b2g4c150", B=2, Hq=8, Hkv=2, C=150, T=4000,
-                                             G=8, L=100, S=32, k=8, n_needles=2, seed=36),
-    "prefill_bf16_g4_k40_c90": LLAMA.replace(name="g4k40", Hq=8, Hkv=2, C=90, T=3000, G=8,
-                                             L=64, S=32, k=40, n_needles=0, seed=37),
+    # GQA 4 with hi/lo query terms and 8 query tiles: the step's two-pass span
+    # filter, with two sequences, and with k a large share of the spans (many
+    # candidates)
+    "prefill_bf16_b2_g4_c1000": LLAMA.replace(name="b2g4c1000", B=2, Hq=4, Hkv=1, C=1000,
+                                              T=4000, G=8, L=100, S=32, k=8, n_needles=2,
+                                              seed=36),
+    "prefill_bf16_g4_k40_c1000": LLAMA.replace(name="g4k40", Hq=8, Hkv=2, C=1000, T=3000, G=8,
+                                               L=64, S=32, k=40, n_needles=0, seed=37),
     "two_level_topk": LLAMA.replace(name="big_ns", Hq=2, Hkv=1, d=64, T=200000, G=32, L=256,
                                     S=8, k=100, n_needles=4, seed=21),
     "batch3_large_s": TINY.replace(name="b3", B=3, Hq=2, Hkv=1, T=5000, G=2, L=40, S=100, k=3,
