@@ -81,9 +81,8 @@ CASES = {
                                               L=256, S=32, k=16, n_needles=3, seed=33),
     "prefill_bf16_b2_c150": LLAMA.replace(name="b2c150", B=2, Hq=4, Hkv=2, C=150, T=4000, G=8,
                                           L=100, S=32, k=8, n_needles=2, seed=35),
-    # GQA 4 with hi/lo query terms and 8 query tiles: the step's two-pass span
-    # filter, with two sequences, and with k a large share of the spans (many
-    # candidates)
+    # GQA 4 with hi/lo query terms and 8 query tiles (four query-slot pairs),
+    # two sequences, and k a large share of the spans
     "prefill_bf16_b2_g4_c1000": LLAMA.replace(name="b2g4c1000", B=2, Hq=4, Hkv=1, C=1000,
                                               T=4000, G=8, L=100, S=32, k=8, n_needles=2,
                                               seed=36),

@@ -876,14 +876,19 @@ static int tc_terms(const Geom &geo) { return geo.g <= 2 ? geo.g : 2; }
 static size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
 // The two-pass filter serves the fused step's query-resident scan with hi/lo
-// query terms when one CTA can rank a head's spans and the chunk has at
-// least 8 query tiles: the key-norm pass reads every middle key once, which
-// halving the products repays only with enough queries per key (at 4 query
-// tiles a 512-query chunk over 128K took 260 instead of 234 us).
+// query terms when one CTA can rank a head's spans and it pays: measured at
+// 8 KV heads, the hi-only pass saves ~22 us per query tile per 2,016 key
+// tiles, the key-norm pass costs ~77 us per 2,016 key tiles, and the exact
+// pass plus the candidate selection ~113 us (they scale with the listed
+// tiles, ~100 per head, not with the context).  So a 2048-query chunk over
+// 256K gains (1.69 -> 1.48 ms), over 64K it loses (~25 us), and so does a
+// 512-query chunk over 128K (260 instead of 234 us).
 static bool filter_eligible(const Geom &geo)
 {
+    const int64_t nqt = (geo.C + kTileN - 1) / kTileN;
+    const int64_t nkt = (geo.M + kTileM - 1) / kTileM;
     return geo.S == 32 && geo.g > 2 && tc_terms(geo) == 2 && geo.NS <= kCandThreads * kCandE &&
-           geo.k > 0 && geo.k < geo.NS && (geo.C + kTileN - 1) / kTileN >= 8;
+           geo.k > 0 && geo.k < geo.NS && nkt * (22 * nqt - 77) > 133 * 2016;
 }
 
 static size_t terms_bytes(const Geom &geo)
