@@ -876,19 +876,26 @@ static int tc_terms(const Geom &geo) { return geo.g <= 2 ? geo.g : 2; }
 static size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
 // The two-pass filter serves the fused step's query-resident scan with hi/lo
-// query terms when one CTA can rank a head's spans and it pays: measured at
-// 8 KV heads, the hi-only pass saves ~22 us per query tile per 2,016 key
-// tiles, the key-norm pass costs ~77 us per 2,016 key tiles, and the exact
-// pass plus the candidate selection ~113 us (they scale with the listed
-// tiles, ~100 per head, not with the context).  So a 2048-query chunk over
-// 256K gains (1.69 -> 1.48 ms), over 64K it loses (~25 us), and so does a
-// 512-query chunk over 128K (260 instead of 234 us).
+// query terms when one CTA can rank a head's spans and it pays.  Fitted to
+// the step at 8 KV heads (costs scale with the heads): the hi-only pass saves
+// ~22 us per query tile per 2,016 key tiles; the key-norm pass costs ~77 us
+// per 2,016 key tiles; the exact pass ~40 + 0.9 k us per 16 query tiles
+// (it scales with the listed tiles, ~1.5 k per head, not with the context);
+// the candidate selection ~13 us.  Measured on a 2048-query chunk over 256K
+// (filter on vs off): k = 64 +198 us, 128 +147, 256 +21, 512 -177, 1024 -486;
+// over 64K with k = 64 -24 us; a 512-query chunk over 128K 260 vs 234 us.
 static bool filter_eligible(const Geom &geo)
 {
-    const int64_t nqt = (geo.C + kTileN - 1) / kTileN;
-    const int64_t nkt = (geo.M + kTileM - 1) / kTileM;
-    return geo.S == 32 && geo.g > 2 && tc_terms(geo) == 2 && geo.NS <= kCandThreads * kCandE &&
-           geo.k > 0 && geo.k < geo.NS && nkt * (22 * nqt - 77) > 133 * 2016;
+    if (!(geo.S == 32 && geo.g > 2 && tc_terms(geo) == 2 && geo.NS <= kCandThreads * kCandE &&
+          geo.k > 0 && geo.k < geo.NS))
+        return false;
+    const double nqt = double((geo.C + kTileN - 1) / kTileN);
+    const double nkt = double((geo.M + kTileM - 1) / kTileM);
+    const double heads = double(geo.B) * geo.Hkv / 8.0;
+    const double gain_us = heads * (22.0 * nqt * nkt / 2016.0 - 77.0 * nkt / 2016.0 -
+                                    nqt / 16.0 * (40.0 + 0.9 * double(geo.k))) -
+                           13.0;
+    return gain_us > 20.0;
 }
 
 static size_t terms_bytes(const Geom &geo)
